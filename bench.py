@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flux|reference]
+
+One step is one pass of the routed prefill hot path over the Qwen3-4B-shaped
+layer workload (B 1, T 32768, Hq 32, Hkv 8, d 128, bf16 N(0,1) with 16 planted
+needles per kv head):
+  flux_route (hidden 32768 x 2560, MLP 5120 -> 512 -> 2, biases put layer 0 on
+  FA and layer 1 on SA) -> flux_build_streaming_mask + flux_build_block_index
+  (block 128, sink 1, window 16) -> flux_attn_prefill for layer 0 (FA) and
+  layer 1 (SA), each reading its routing bit on the device.
+value = TFLOP/s over computed (query, key) pairs of both layers (4 d FLOPs per
+pair per head) / step time.  The decode half of the metric (KV GB/s) is timed
+in the same run on the 36-layer Qwen3-4B-shaped decode workload (batch 16, KV
+131072 + step, 18 FA / 18 SA layers, 64 steps) and reported under "decode".
+
+Every input is seeded and synthetic; every timed input (640 MB for prefill,
+17 GB of KV for decode) is larger than the 126 MB L2, so no flush is needed.
+Multi-GPU: the units are independent (no exchange), so each rank runs its own
+replica of the step (weak scaling) and rank 0 reports the max time.
+
+--impl reference times the oracle (plain fp64 C, OpenMP) on the host cores on
+a bounded sample of the same workload, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+T, HQ, HKV, D = 32768, 32, 8, 128
+HD, H1 = 2560, 512
+BLOCK, SINK, WIN = 128, 1, 16
+DEC_B, DEC_S, DEC_LAYERS, DEC_STEPS = 16, 131072, 36, 64
+
+
+def causal_pairs_fa(T):
+    return T * (T + 1) // 2
+
+
+def pairs_sa(T, block, sink, W):
+    """(query, key) pairs visible under the sink + window mask (diagonal tiles causal)."""
+    nb = (T + block - 1) // block
+    total = 0
+    for i in range(nb):
+        q0, q1 = i * block, min(T, (i + 1) * block)
+        for j in range(i + 1):
+            if not (j < sink or j >= i - W + 1):
+                continue
+            k0, k1 = j * block, min(T, (j + 1) * block)
+            if j < i:
+                total += (q1 - q0) * (k1 - k0)
+            else:
+                n = q1 - q0
+                total += n * (n + 1) // 2
+    return total
+
+
+def sa_decode_tokens(s, block, sink, W):
+    n_sink = min(sink * block, s)
+    nbs = -(-s // block)
+    win_start = max(n_sink, max(0, nbs - W) * block)
+    return n_sink + (s - win_start)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if not self.path or not os.path.exists(self.path):
+            return out
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return out
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        out.update(sm_mhz=statistics.median(sm) if sm else None,
+                   sm_max_mhz=max(mx) if mx else None, reasons=sorted(reasons),
+                   samples=len(rows))
+        return out
+
+
+# --------------------------------------------------------------------------- flux arm
+
+class PrefillWorkload:
+    def __init__(self, ctx, seed, dev):
+        import torch
+        from sparse_attention_flux_b200 import synth
+        self.ctx, self.dev = ctx, dev
+        g = torch.Generator(device=dev)
+        q, k, v = synth.attention_inputs(1, T, HQ, HKV, D, seed)
+        self.needles = synth.plant_needles_np(q, k, seed)
+        self.q_h = synth.torch_from_bits(q).pin_memory()
+        self.k_h = synth.torch_from_bits(k).pin_memory()
+        self.v_h = synth.torch_from_bits(v).pin_memory()
+        self.q, self.k, self.v = (x.to(dev) for x in (self.q_h, self.k_h, self.v_h))
+        hidden, W1, b1, W2, b2 = synth.router_inputs(T, HD, H1, 2, seed + 50)
+        b2[:] = np.array([4.0, -4.0], np.float32)   # layer 0 -> FA, layer 1 -> SA
+        self.hidden_h = synth.torch_from_bits(hidden).pin_memory()
+        self.hidden = self.hidden_h.to(dev)
+        self.W1, self.b1, self.W2, self.b2 = (torch.from_numpy(x).to(dev) for x in (W1, b1, W2, b2))
+        self.mode = torch.zeros(2, dtype=torch.uint8, device=dev)
+        self.nb = T // BLOCK
+        self.mask = torch.empty((self.nb, self.nb), dtype=torch.uint8, device=dev)
+        self.row_ptr = torch.empty(self.nb + 1, dtype=torch.int32, device=dev)
+        self.col = torch.empty(self.nb * (SINK + WIN), dtype=torch.int32, device=dev)
+        self.o = [torch.empty_like(self.q) for _ in range(2)]
+        self.o_h = [torch.empty_like(self.q_h).pin_memory() for _ in range(2)]
+        self.flops_fa = 4.0 * D * causal_pairs_fa(T) * HQ
+        self.flops_sa = 4.0 * D * pairs_sa(T, BLOCK, SINK, WIN) * HQ
+        self.flops = self.flops_fa + self.flops_sa
+        self.launches = 2 + 1 + 3 + 2
+        self.scale = 1.0 / math.sqrt(D)
+
+    def step(self, events=None):
+        c = self.ctx
+        c.route(self.hidden, self.W1, self.b1, self.W2, self.b2, 0.5, self.mode)
+        c.build_streaming_mask(self.nb, self.nb, SINK, WIN, self.mask)
+        c.build_block_index(self.mask, self.row_ptr, self.col)
+        for layer in (0, 1):
+            if events:
+                events[layer][0].record()
+            c.attn_prefill(self.q, self.k, self.v, self.o[layer], self.scale, layer_mode=self.mode,
+                           layer=layer, row_ptr=self.row_ptr, col=self.col, block=BLOCK)
+            if events:
+                events[layer][1].record()
+
+    def step_e2e(self):
+        # Host buffers in, host buffers out: the copies are inside the timed region.
+        for dst, src in ((self.q, self.q_h), (self.k, self.k_h), (self.v, self.v_h),
+                         (self.hidden, self.hidden_h)):
+            dst.copy_(src, non_blocking=True)
+        self.step()
+        for l in (0, 1):
+            self.o_h[l].copy_(self.o[l], non_blocking=True)
+
+    @property
+    def h2d_bytes(self):
+        return sum(x.numel() * 2 for x in (self.q_h, self.k_h, self.v_h, self.hidden_h))
+
+    @property
+    def d2h_bytes(self):
+        return sum(x.numel() * 2 for x in self.o_h)
+
+
+class DecodeWorkload:
+    def __init__(self, ctx, seed, dev, steps):
+        import torch
+        from sparse_attention_flux_b200 import synth
+        self.ctx, self.dev, self.steps = ctx, dev, steps
+        self.S_max = DEC_S + steps
+        shape = (DEC_B, self.S_max, HKV, D)
+        # 18 FA layers alias onto 2 physical caches (each 8.6 GB, far above L2);
+        # SA layers share one cache and touch only sink + window blocks.
+        self.fa_caches = [(synth.torch_normal_bf16(shape, seed + 10 * i + 1, dev),
+                           synth.torch_normal_bf16(shape, seed + 10 * i + 2, dev)) for i in range(2)]
+        self.sa_cache = self.fa_caches[0]
+        self.mode = torch.from_numpy(synth.layer_mode_choice(DEC_LAYERS, DEC_LAYERS // 2, seed)).to(dev)
+        self.mode_h = self.mode.cpu().numpy()
+        self.q = synth.torch_normal_bf16((DEC_B, HQ, D), seed + 99, dev)
+        self.o = torch.empty_like(self.q)
+        self.seqlens = [torch.full((DEC_B,), DEC_S + s, dtype=torch.int32, device=dev)
+                        for s in range(steps)]
+        self.scale = 1.0 / math.sqrt(D)
+        kv_row = HKV * D * 2 * 2
+        self.bytes_fa = sum(DEC_B * (DEC_S + s) * kv_row for s in range(steps)) / steps
+        self.bytes_sa = sum(DEC_B * sa_decode_tokens(DEC_S + s, BLOCK, SINK, WIN) * kv_row
+                            for s in range(steps)) / steps
+        n_fa = int(self.mode_h.sum())
+        self.bytes_per_step = n_fa * self.bytes_fa + (DEC_LAYERS - n_fa) * self.bytes_sa
+        self.launches = DEC_LAYERS
+
+    def step(self, s, fa_events=None):
+        c = self.ctx
+        fa_i = 0
+        for layer in range(DEC_LAYERS):
+            if self.mode_h[layer]:
+                kc, vc = self.fa_caches[fa_i % 2]
+                fa_i += 1
+            else:
+                kc, vc = self.sa_cache
+            if fa_events is not None and self.mode_h[layer] and fa_i == 1:
+                fa_events[0].record()
+            c.attn_decode(self.q, kc, vc, self.seqlens[s], self.o, self.scale, layer_mode=self.mode,
+                          layer=layer, sink_blocks=SINK, window_blocks=WIN, block=BLOCK)
+            if fa_events is not None and self.mode_h[layer] and fa_i == 1:
+                fa_events[1].record()
+
+
+def run_flux(args, rank, world, dev_index):
+    import torch
+    import torch.distributed as dist
+    from sparse_attention_flux_b200.flux import Context
+
+    torch.cuda.set_device(dev_index)
+    dev = torch.device("cuda", dev_index)
+    peaks, peak_src = load_peaks()
+    ctx = Context(dev_index, 512 << 20)
+    from sparse_attention_flux_b200 import synth
+    wl = PrefillWorkload(ctx, synth.seed_for(1) + 1000 * rank, dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        wl.step()
+    ctx.check()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(2)]
+    fa_ms, sa_ms = [], []
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev_index) as clk:
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(args.steps):
+            wl.step(ev)
+            # per-kernel durations from events on the launching (current) stream
+            stop.record()
+            stop.synchronize()
+            fa_ms.append(ev[0][0].elapsed_time(ev[0][1]))
+            sa_ms.append(ev[1][0].elapsed_time(ev[1][1]))
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = start.elapsed_time(stop)
+    ctx.check()
+    clocks = clk.summary()
+    total_ms = max_over_ranks(total_ms)
+    ms_per_step = total_ms / args.steps
+    value = wl.flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # e2e: host buffers in and out through the same public API
+    for _ in range(max(1, args.warmup // 2)):
+        wl.step_e2e()
+    torch.cuda.synchronize()
+    barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    e2e_steps = max(2, args.steps // 2)
+    for _ in range(e2e_steps):
+        wl.step_e2e()
+    s1.record()
+    s1.synchronize()
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / e2e_steps)
+    e2e_value = wl.flops * world / (e2e_ms * 1e-3) / 1e12
+
+    h2d_bytes, d2h_bytes, launches = wl.h2d_bytes, wl.d2h_bytes, wl.launches * args.steps
+    fa_avg = statistics.mean(fa_ms)
+    sa_avg = statistics.mean(sa_ms)
+    peak_t = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    fa_tflops = wl.flops_fa / (fa_avg * 1e-3) / 1e12
+    sa_tflops = wl.flops_sa / (sa_avg * 1e-3) / 1e12
+
+    # decode half of the metric
+    del wl
+    torch.cuda.empty_cache()
+    dec = None
+    if not args.no_decode:
+        dw = DecodeWorkload(ctx, synth.seed_for(3) + 1000 * rank, dev, args.decode_steps)
+        for s in range(min(3, dw.steps)):
+            dw.step(s)
+        ctx.check()
+        fev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        fa_dec_ms = []
+        barrier()
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record()
+        for s in range(dw.steps):
+            dw.step(s, fev)
+            fev[1].synchronize()
+            fa_dec_ms.append(fev[0].elapsed_time(fev[1]))
+        d1.record()
+        d1.synchronize()
+        ctx.check()
+        dec_ms = max_over_ranks(d0.elapsed_time(d1) / dw.steps)
+        dec_gbs = dw.bytes_per_step * world / (dec_ms * 1e-3) / 1e9
+        fa_dec_avg = statistics.mean(fa_dec_ms)
+        fa_dec_gbs = dw.bytes_fa / (fa_dec_avg * 1e-3) / 1e9
+        dec = {
+            "workload": "qwen3-4b-36L-routed-decode: B 16, KV 131072+step, 18 FA / 18 SA, "
+                        f"{dw.steps} steps",
+            "value": round(dec_gbs, 1), "unit": "GB/s (KV bytes that must be read)",
+            "ms_per_step": round(dec_ms, 4), "gpu_launches_per_step": dw.launches,
+            "frac_of_hbm": round(dec_gbs / peaks["hbm_gbs"], 4),
+            "fa_layer": {"GB/s": round(fa_dec_gbs, 1), "ms": round(fa_dec_avg, 4),
+                         "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4)},
+        }
+        roof_dec = {"bound": "hbm", "achieved": round(fa_dec_gbs, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4),
+                    "traffic": None, "kernel": "decode_kernel<128,4> (FA layer)"}
+        dec["roofline"] = roof_dec
+        del dw
+    ctx.close()
+
+    line = {
+        "metric": "routed-attn prefill TFLOP/s & decode KV GB/s at 1 B200; % of roofline",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "qwen3-4b-layer-routed-prefill: B 1, T 32768, Hq 32, Hkv 8, d 128, "
+                               "needles; router 32768x2560 -> MLP 5120-512-2 (layer0 FA, layer1 SA); "
+                               "SA block 128, sink 1, window 16",
+                   "l2": "inputs larger than L2 (640 MB prefill, 17 GB decode KV); no flush",
+                   "parallelism": f"replicas x{world} (no exchange)"},
+        "roofline": {"bound": "tensor", "achieved": round(fa_tflops, 1), "peak": peak_t,
+                     "unit": "TFLOP/s", "frac": round(fa_tflops / peak_t, 4), "traffic": None,
+                     "kernel": "prefill_kernel<128> (FA layer)",
+                     "peak_source": f"{peak_src} bf16_tflops_sustained"},
+        "sa_prefill": {"TFLOP/s": round(sa_tflops, 1), "ms": round(sa_avg, 4),
+                       "frac": round(sa_tflops / peak_t, 4)},
+        "fa_prefill": {"TFLOP/s": round(fa_tflops, 1), "ms": round(fa_avg, 4)},
+        "decode": dec,
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
+                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "context": "pages: up to 2.8x prefill / 2.0x decode speedup vs FA baseline, hardware not "
+                   "stated on the pages",
+    }
+    return line
+
+
+def cpu_baseline(seconds_budget=15.0):
+    """The oracle, as it stands, on a bounded sample of the same prefill workload."""
+    import oracle
+    from sparse_attention_flux_b200 import synth
+    seed = synth.seed_for(1)
+    q, k, v = synth.attention_inputs(1, T, HQ, HKV, D, seed)
+    synth.plant_needles_np(q, k, seed)
+    scale = 1.0 / math.sqrt(D)
+    nb = T // BLOCK
+    m = oracle.streaming_mask(nb, nb, SINK, WIN)
+    r = synth.rng(seed + 9)
+    # Sample rows uniformly; time FA rows until the budget is half spent, then SA rows.
+    done_pairs, t_used, n_rows = 0, 0.0, 0
+    for sparse in (False, True):
+        budget = seconds_budget / 2
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < budget:
+            rows = np.stack([np.zeros(64, np.int32), r.integers(0, HQ, 64).astype(np.int32),
+                             r.integers(0, T, 64).astype(np.int32)], 1)
+            oracle.attn_prefill(q, k, v, scale, block_mask=m if sparse else None, block=BLOCK,
+                                rows=rows)
+            for t in rows[:, 2]:
+                if sparse:
+                    i = t // BLOCK
+                    done_pairs += sum(min(BLOCK, t + 1 - j * BLOCK) for j in range(i + 1)
+                                      if (j < SINK or j >= i - WIN + 1))
+                else:
+                    done_pairs += t + 1
+            n_rows += 64
+        t_used += time.perf_counter() - t0
+    tflops = 4.0 * D * done_pairs / t_used / 1e12
+    return {"value": tflops, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n_rows} uniformly sampled query rows (half FA, half SA) of the T=32768 "
+                      f"layer, {t_used:.1f} s; FLOPs counted like the GPU's (4 d per visible pair)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["flux", "reference"], default="flux")
+    ap.add_argument("--decode-steps", type=int, default=DEC_STEPS)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        base = cpu_baseline(args.cpu_seconds)
+        per_step_s = args.cpu_seconds
+        line = {"metric": "routed-attn prefill TFLOP/s & decode KV GB/s at 1 B200; % of roofline",
+                "impl": "reference", "value": base["value"], "unit": "TFLOP/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": per_step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": "qwen3-4b-layer-routed-prefill: B 1, T 32768, Hq 32, Hkv 8, "
+                                       "d 128 (sampled rows)"},
+                "cpu_baseline": base,
+                "e2e": {"value": base["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    line = run_flux(args, rank, world, local)
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,186 @@
+/*
+ * flux.h -- C ABI of the B200 (sm_100a) routed-attention library (libflux.so).
+ *
+ * Flux Attention ("Flux Attention: Context-Aware Hybrid Attention for
+ * Efficient LLMs Inference", arXiv 2604.07394) puts a small Layer Router in
+ * front of a frozen LLM.  The router looks at the prompt once, at prefill,
+ * and sends every layer either to Full Attention (FA: exact causal softmax
+ * attention) or to Sparse Attention (SA: block-sparse attention over a sink +
+ * local-window block mask).  The decision is reused for every decode step,
+ * and SA layers read only the minimal KV.  This header exposes that hot path:
+ *
+ *   flux_route                 pool + MLP + hard threshold  -> layer_mode[L]
+ *   flux_build_streaming_mask  sink + window block mask     -> mask[nqb][nkb]
+ *   flux_build_block_index     block mask                   -> CSR row_ptr/col
+ *   flux_attn_prefill          one layer, FA or SA per layer_mode[layer]
+ *   flux_attn_decode           one layer, one new token per sequence
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the
+ *     library never frees or keeps it beyond the call's stream work.
+ *   - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and returns an int status.  Host-side argument
+ *     checks happen before any launch; on failure nothing is launched.
+ *   - Device-side checks (seqlens beyond capacity, CSR entries out of range,
+ *     a bounded wait that ran out) set the context's device error word and
+ *     zero the affected outputs; flux_ctx_check() reports it.
+ *   - The routing bit is read ON THE DEVICE (layer_mode[layer]; 1 = FA,
+ *     0 = SA), so routing and attention chain on one stream with no host sync.
+ *   - A flux_ctx owns the only memory the library allocates (a workspace for
+ *     split-KV decode partials and router intermediates, and the error word).
+ *     Calls that share a ctx must not overlap in time on different streams.
+ *   - flux_last_error() describes the last failure of the calling thread.
+ */
+#ifndef FLUX_H
+#define FLUX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLUX_ABI_VERSION 1
+
+/* Status codes. */
+#define FLUX_OK                0
+#define FLUX_ERR_INVALID_ARG  -1  /* null pointer, negative size, bad threshold ...        */
+#define FLUX_ERR_SHAPE        -2  /* sizes inconsistent or beyond capacity / workspace      */
+#define FLUX_ERR_UNSUPPORTED  -3  /* e.g. head_dim not 64/128, Hq % Hkv != 0, block size   */
+#define FLUX_ERR_CUDA         -4  /* a CUDA runtime call failed (launch, memcpy, ...)       */
+#define FLUX_ERR_TIMEOUT      -5  /* a bounded device-side wait ran out (device error word) */
+#define FLUX_ERR_DEVICE_CHECK -6  /* a device-side range check failed (device error word)   */
+
+typedef struct flux_ctx flux_ctx;
+typedef void* flux_stream_t; /* cudaStream_t */
+
+/* ABI version (FLUX_ABI_VERSION). */
+int flux_version(void);
+
+/* Message for the calling thread's last failed call ("" if none). */
+const char* flux_last_error(void);
+
+/* Create a context on CUDA device `device`, allocating `workspace_bytes` of
+ * device workspace (0 = a default of 64 MiB) plus the device error word.
+ * The workspace holds split-KV decode partials and router intermediates; use
+ * flux_decode_workspace_bytes() to size it for a decode shape.  The ctx is
+ * bound to `device`; calls through it must run with that device current. */
+int flux_ctx_create(flux_ctx** ctx, int device, size_t workspace_bytes);
+
+/* Free the context's device memory.  Pending work on any stream that used the
+ * ctx must be complete. */
+int flux_ctx_destroy(flux_ctx* ctx);
+
+/* Synchronize `stream`, read and clear the device error word.  Returns
+ * FLUX_OK, FLUX_ERR_TIMEOUT, FLUX_ERR_DEVICE_CHECK or FLUX_ERR_CUDA. */
+int flux_ctx_check(flux_ctx* ctx, flux_stream_t stream);
+
+/* Spin limit of every bounded device-side wait, in milliseconds (default
+ * 2000).  A wait that runs out sets the error word and makes the kernel
+ * release its resources and return. */
+int flux_ctx_set_spin_limit_ms(flux_ctx* ctx, int ms);
+
+/* --------------------------------------------------------------------------
+ * Layer Router (gist.science summary "Flux Attention", section 2
+ * "Methodology": "Layer Router" pools the first and last 100 prompt tokens
+ * and runs a context-encoder MLP; "switch to hard routing" thresholds the
+ * soft weight to 0/1 at inference; "efficient deployment" routes once, at
+ * prefill).
+ *   hidden     [T, Hd] bf16, row-major: the prompt's hidden states.
+ *   n_pool     rows pooled on each side (100 on the pages); each side uses
+ *              n = min(n_pool, T) rows, so the windows overlap when T < 2 n.
+ *   p          = [mean(hidden[0:n]), mean(hidden[T-n:T])]      (2*Hd, fp32)
+ *   W1 [H1, 2*Hd], b1 [H1], W2 [L, H1], b2 [L]: fp32, row-major.
+ *   z          = W2 relu(W1 p + b1) + b2;  r = sigmoid(z)
+ *   layer_mode [L] uint8 out: 1 (FA) iff r > thresh, else 0 (SA); a tie is SA.
+ *   score      [L] fp32 out (optional, may be NULL): r.
+ * Uses 4 * (2*Hd + H1) + 64 bytes of the ctx workspace.
+ * Errors: INVALID_ARG for null required pointers, sizes <= 0, thresh not
+ * finite; SHAPE if the workspace is too small. */
+int flux_route(flux_ctx* ctx, const uint16_t* hidden, int T, int Hd, int n_pool,
+               const float* W1, const float* b1, int H1,
+               const float* W2, const float* b2, int L,
+               float thresh, uint8_t* layer_mode, float* score, flux_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * SA block mask: attention sinks plus a local window of recent blocks (the
+ * block-sparse SA of the model card "Flux Attention: Qwen3-4B", "Sample
+ * Usage"; SA keeps only the minimal KV, gist.science summary section 2).
+ *   block_mask [nqb, nkb] uint8 out, row-major:
+ *     mask[i][j] = (j <= i) && (j < sink_blocks || j >= i - window_blocks + 1)
+ *   The window counts the diagonal block.  sink_blocks >= 0, window_blocks >= 1. */
+int flux_build_streaming_mask(int nqb, int nkb, int sink_blocks, int window_blocks,
+                              uint8_t* block_mask, flux_stream_t stream);
+
+/* Compressed block-index list of a block mask (the form the prefill kernel
+ * walks, so that skipped blocks cost no memory traffic).
+ *   block_mask [nqb, nkb] uint8 in (nonzero = keep).
+ *   row_ptr [nqb + 1] int32 out; row_ptr[nqb] = nnz.
+ *   col [cap] int32 out: for each q-block i, the ascending kept kv blocks in
+ *   col[row_ptr[i] .. row_ptr[i+1]).
+ * If nnz > cap, nothing beyond cap is written and the device error word is
+ * set (flux_ctx_check -> FLUX_ERR_DEVICE_CHECK).  Uses 4 * nqb bytes of the
+ * ctx workspace. */
+int flux_build_block_index(flux_ctx* ctx, const uint8_t* block_mask, int nqb, int nkb,
+                           int32_t* row_ptr, int32_t* col, int cap, flux_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Prefill attention for one layer (arXiv abstract: FA = exact causal full
+ * attention; SA = sparse attention; routing is per layer).
+ *   q [B, T, Hq, d], k and v [B, T, Hkv, d]: bf16, contiguous.
+ *   o [B, T, Hq, d] bf16 out.  lse [B, Hq, T] fp32 out (optional): natural-log
+ *   sum of exp of the scaled scores; -inf for a row with no visible key.
+ *   Query head h reads kv head h / (Hq / Hkv).
+ *   layer_mode: device uint8 array; layer_mode[layer] = 1 -> FA (every key
+ *   u <= t), 0 -> SA (u <= t and the block pair (t / block, u / block) is in
+ *   the CSR list).  layer_mode == NULL means FA.
+ *   row_ptr/col: the CSR list from flux_build_block_index over nqb >=
+ *   ceil(T / block) q-blocks; required unless layer_mode == NULL.
+ *   block: 64 or a multiple of 128.  d: 64 or 128.  scale: score scale
+ *   (1/sqrt(d) for the models on the pages).
+ * Runs the tcgen05/TMEM/TMA flash-attention kernel; skipped blocks are never
+ * loaded.  Errors: UNSUPPORTED for other d or block, or Hq % Hkv != 0; SHAPE
+ * for T < 1, nqb too small, or sizes whose tensor maps cannot be encoded. */
+int flux_attn_prefill(flux_ctx* ctx, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      uint16_t* o, float* lse, int B, int T, int Hq, int Hkv, int d,
+                      const uint8_t* layer_mode, int layer,
+                      const int32_t* row_ptr, const int32_t* col, int nqb, int block,
+                      float scale, flux_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Decode attention for one layer and one new token per sequence (gist.science
+ * summary section 2, "efficient deployment": the prefill routing bit is
+ * reused; SA layers read only the sink blocks and the last W blocks).
+ *   q [B, Hq, d] bf16: the query of the token at position seqlens[b] - 1.
+ *   k_cache, v_cache [B, S_max, Hkv, d] bf16; the caller has already appended
+ *   the new token's k/v, so positions 0 .. seqlens[b]-1 are valid.
+ *   seqlens [B] int32 device array, 0 <= seqlens[b] <= S_max (checked on the
+ *   device; a bad value zeroes that sequence's output and sets the error word).
+ *   o [B, Hq, d] bf16 out; lse [B, Hq] fp32 out (optional).
+ *   layer_mode[layer]: 1 -> FA over all u < s; 0 -> SA over the tokens in
+ *   blocks j < sink_blocks or j >= ceil(s / block) - window_blocks.
+ *   layer_mode == NULL means FA.
+ * Split-KV: each CTA streams one chunk of one (sequence, kv head) and serves
+ * all Hq/Hkv query heads of the group from that single read; the last CTA of
+ * the group (atomic ticket, no spin) merges the partials.  Partials live in
+ * the ctx workspace (flux_decode_workspace_bytes).  Supported: d 64/128,
+ * Hq/Hkv in {1, 2, 4}.  Calls sharing a ctx must not overlap in time. */
+int flux_attn_decode(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_cache,
+                     const uint16_t* v_cache, int S_max, const int32_t* seqlens,
+                     uint16_t* o, float* lse, int B, int Hq, int Hkv, int d,
+                     const uint8_t* layer_mode, int layer,
+                     int sink_blocks, int window_blocks, int block, float scale,
+                     flux_stream_t stream);
+
+/* Workspace bytes flux_attn_decode needs on this ctx's device for this shape
+ * and SA window (host-only query; no device work). */
+int flux_decode_workspace_bytes(flux_ctx* ctx, int B, int Hq, int Hkv, int d, int S_max,
+                                int sink_blocks, int window_blocks, int block, size_t* bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLUX_H */

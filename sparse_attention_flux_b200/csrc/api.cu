@@ -1,0 +1,363 @@
+// api.cu -- the C ABI of libflux (declared in include/flux.h): context and
+// workspace management, host-side argument checks, TMA tensor-map encoding
+// and the kernel launches.  No torch types cross this boundary.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "flux.h"
+#include "kernels.h"
+
+struct flux_ctx {
+  int device;
+  int num_sms;
+  void* workspace;        // scratch shared by the calls (they must not overlap in time)
+  size_t workspace_bytes;
+  int* tickets;           // [kMaxTickets + 1] ints, zero between calls; last one: router
+  int* err;               // device error word
+  long long spin_ns;
+};
+
+namespace {
+
+constexpr int kMaxTickets = 1 << 16;
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(FLUX_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- TMA descriptor encoding through the driver entry point (no -lcuda)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+EncodeTiledFn encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+// A bf16 tensor [d3][d2][d1][d0] (d0 innermost), boxes of box0 x 1 x box2 x 1
+// with the 128-byte swizzle; out-of-range rows read as zero.
+int make_map_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                uint64_t d3, uint32_t box0, uint32_t box2) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(FLUX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t gdim[4] = {d0, d1, d2, d3};
+  const cuuint64_t gstride[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  const cuuint32_t box[4] = {box0, 1, box2, 1};
+  const cuuint32_t estride[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gdim,
+                         gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FLUX_ERR_SHAPE, "tensor map encoding failed (CUresult %d)", r);
+  return FLUX_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+flux::DevStatus status_of(const flux_ctx* c) { return flux::DevStatus{c->err, c->spin_ns}; }
+
+}  // namespace
+
+extern "C" {
+
+int flux_version(void) { return FLUX_ABI_VERSION; }
+
+const char* flux_last_error(void) { return g_last_error.c_str(); }
+
+int flux_ctx_create(flux_ctx** out, int device, size_t workspace_bytes) {
+  if (!out) return fail(FLUX_ERR_INVALID_ARG, "flux_ctx_create: null output pointer");
+  *out = nullptr;
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
+  if (device < 0 || device >= ndev) return fail(FLUX_ERR_INVALID_ARG, "no CUDA device %d", device);
+  if ((e = cudaSetDevice(device)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  cudaDeviceProp prop;
+  if ((e = cudaGetDeviceProperties(&prop, device)) != cudaSuccess)
+    return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10)
+    return fail(FLUX_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                device, prop.major, prop.minor);
+  flux_ctx* c = static_cast<flux_ctx*>(calloc(1, sizeof(flux_ctx)));
+  if (!c) return fail(FLUX_ERR_INVALID_ARG, "out of host memory");
+  c->device = device;
+  c->num_sms = prop.multiProcessorCount;
+  c->workspace_bytes = workspace_bytes ? workspace_bytes : (size_t(64) << 20);
+  c->spin_ns = 2000LL * 1000000LL;
+  if (const char* s = getenv("FLUX_SPIN_LIMIT_MS")) {
+    const long long ms = atoll(s);
+    if (ms > 0) c->spin_ns = ms * 1000000LL;
+  }
+  if ((e = cudaMalloc(&c->workspace, c->workspace_bytes)) != cudaSuccess ||
+      (e = cudaMalloc(reinterpret_cast<void**>(&c->tickets), (kMaxTickets + 1) * sizeof(int))) !=
+          cudaSuccess ||
+      (e = cudaMalloc(reinterpret_cast<void**>(&c->err), sizeof(int))) != cudaSuccess ||
+      (e = cudaMemset(c->tickets, 0, (kMaxTickets + 1) * sizeof(int))) != cudaSuccess ||
+      (e = cudaMemset(c->err, 0, sizeof(int))) != cudaSuccess ||
+      (e = cudaDeviceSynchronize()) != cudaSuccess) {
+    cudaFree(c->workspace);
+    cudaFree(c->tickets);
+    cudaFree(c->err);
+    free(c);
+    return cuda_fail(e, "flux_ctx_create: device allocation");
+  }
+  *out = c;
+  return FLUX_OK;
+}
+
+int flux_ctx_destroy(flux_ctx* c) {
+  if (!c) return fail(FLUX_ERR_INVALID_ARG, "flux_ctx_destroy: null ctx");
+  cudaFree(c->workspace);
+  cudaFree(c->tickets);
+  cudaFree(c->err);
+  free(c);
+  return FLUX_OK;
+}
+
+int flux_ctx_set_spin_limit_ms(flux_ctx* c, int ms) {
+  if (!c || ms <= 0) return fail(FLUX_ERR_INVALID_ARG, "flux_ctx_set_spin_limit_ms: bad argument");
+  c->spin_ns = static_cast<long long>(ms) * 1000000LL;
+  return FLUX_OK;
+}
+
+int flux_ctx_check(flux_ctx* c, flux_stream_t stream) {
+  if (!c) return fail(FLUX_ERR_INVALID_ARG, "flux_ctx_check: null ctx");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "flux_ctx_check: stream synchronize");
+  int word = 0;
+  if ((e = cudaMemcpy(&word, c->err, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "flux_ctx_check: read error word");
+  if (word == flux::DEV_OK) return FLUX_OK;
+  // Clear the word and any ticket an aborted kernel left behind.
+  cudaMemset(c->err, 0, sizeof(int));
+  cudaMemset(c->tickets, 0, (kMaxTickets + 1) * sizeof(int));
+  cudaDeviceSynchronize();
+  switch (word) {
+    case flux::DEV_ERR_TIMEOUT:
+      return fail(FLUX_ERR_TIMEOUT, "a bounded device-side wait ran out");
+    case flux::DEV_ERR_SEQLEN:
+      return fail(FLUX_ERR_DEVICE_CHECK, "seqlens entry outside [0, S_max]");
+    case flux::DEV_ERR_CSR:
+      return fail(FLUX_ERR_DEVICE_CHECK, "block-index list entry out of range");
+    case flux::DEV_ERR_CAPACITY:
+      return fail(FLUX_ERR_DEVICE_CHECK, "block-index nnz exceeds the col capacity");
+    default:
+      return fail(FLUX_ERR_DEVICE_CHECK, "device error word %d", word);
+  }
+}
+
+int flux_route(flux_ctx* c, const uint16_t* hidden, int T, int Hd, int n_pool, const float* W1,
+               const float* b1, int H1, const float* W2, const float* b2, int L, float thresh,
+               uint8_t* layer_mode, float* score, flux_stream_t stream) {
+  if (!c || !hidden || !W1 || !b1 || !W2 || !b2 || !layer_mode)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_route: null pointer argument");
+  if (T < 1 || Hd < 1 || n_pool < 1 || H1 < 1 || L < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_route: sizes must be positive");
+  if (!(thresh == thresh) || thresh > 3.0e38f || thresh < -3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_route: thresh must be finite");
+  if (!aligned16(hidden) || !aligned16(W1))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_route: hidden and W1 must be 16-byte aligned");
+  const size_t need = flux::route_workspace_bytes(Hd, H1);
+  if (need > c->workspace_bytes)
+    return fail(FLUX_ERR_SHAPE, "flux_route: workspace %zu < %zu bytes", c->workspace_bytes, need);
+  flux::RouteLaunch p;
+  p.hidden = hidden;
+  p.T = T;
+  p.Hd = Hd;
+  p.n_pool = n_pool;
+  p.W1 = W1;
+  p.b1 = b1;
+  p.H1 = H1;
+  p.W2 = W2;
+  p.b2 = b2;
+  p.L = L;
+  p.thresh = thresh;
+  p.layer_mode = layer_mode;
+  p.score = score;
+  p.pooled = static_cast<float*>(c->workspace);
+  p.hidden1 = p.pooled + 2 * Hd;
+  p.ticket = c->tickets + kMaxTickets;
+  const cudaError_t e = flux::launch_route(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_route: launch");
+}
+
+int flux_build_streaming_mask(int nqb, int nkb, int sink_blocks, int window_blocks,
+                              uint8_t* block_mask, flux_stream_t stream) {
+  if (!block_mask) return fail(FLUX_ERR_INVALID_ARG, "flux_build_streaming_mask: null mask");
+  if (nqb < 1 || nkb < 1 || sink_blocks < 0 || window_blocks < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_build_streaming_mask: bad sizes");
+  const cudaError_t e = flux::launch_streaming_mask(nqb, nkb, sink_blocks, window_blocks,
+                                                    block_mask, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_build_streaming_mask: launch");
+}
+
+int flux_build_block_index(flux_ctx* c, const uint8_t* block_mask, int nqb, int nkb,
+                           int32_t* row_ptr, int32_t* col, int cap, flux_stream_t stream) {
+  if (!c || !block_mask || !row_ptr || !col)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_build_block_index: null pointer argument");
+  if (nqb < 1 || nkb < 1 || cap < 0)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_build_block_index: bad sizes");
+  if (static_cast<size_t>(nqb) * sizeof(int32_t) > c->workspace_bytes)
+    return fail(FLUX_ERR_SHAPE, "flux_build_block_index: workspace too small");
+  const cudaError_t e = flux::launch_block_index(block_mask, nqb, nkb, row_ptr, col, cap,
+                                                 static_cast<int32_t*>(c->workspace), c->err,
+                                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_build_block_index: launch");
+}
+
+int flux_attn_prefill(flux_ctx* c, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      uint16_t* o, float* lse, int B, int T, int Hq, int Hkv, int d,
+                      const uint8_t* layer_mode, int layer, const int32_t* row_ptr,
+                      const int32_t* col, int nqb, int block, float scale,
+                      flux_stream_t stream) {
+  if (!c || !q || !k || !v || !o) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: null tensor");
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill: sizes must be positive");
+  if (d != 64 && d != 128)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill: head_dim %d (supported: 64, 128)", d);
+  if (Hq % Hkv != 0)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill: Hq %% Hkv != 0 (%d, %d)", Hq, Hkv);
+  if (block != 64 && (block < 128 || block % 128 != 0))
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill: block %d (64 or a multiple of 128)",
+                block);
+  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: scale must be finite and positive");
+  if (layer_mode) {
+    if (layer < 0) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: negative layer");
+    if (!row_ptr || !col)
+      return fail(FLUX_ERR_INVALID_ARG,
+                  "flux_attn_prefill: row_ptr/col are required when layer_mode is given");
+    if (nqb < (T + block - 1) / block)
+      return fail(FLUX_ERR_SHAPE, "flux_attn_prefill: nqb %d < ceil(T / block) = %d", nqb,
+                  (T + block - 1) / block);
+  }
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: tensors must be 16-byte aligned");
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  flux::PrefillLaunch p;
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.block = block;
+  p.nqb = layer_mode ? nqb : 0;
+  p.scale = scale;
+  p.layer_mode = layer_mode;
+  p.layer = layer;
+  p.row_ptr = row_ptr;
+  p.col = col;
+  p.o = o;
+  p.lse = lse;
+  p.st = status_of(c);
+  const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill: launch");
+}
+
+int flux_decode_workspace_bytes(flux_ctx* c, int B, int Hq, int Hkv, int d, int S_max,
+                                int sink_blocks, int window_blocks, int block, size_t* bytes) {
+  if (!c || !bytes || B < 1 || Hq < 1 || Hkv < 1 || d < 1 || S_max < 1 || block < 1 ||
+      sink_blocks < 0 || window_blocks < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_decode_workspace_bytes: bad arguments");
+  int ns, cfa, csa;
+  flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, c->num_sms, &ns, &cfa, &csa);
+  *bytes = flux::decode_workspace_bytes(B, Hq, Hkv, d, ns);
+  return FLUX_OK;
+}
+
+int flux_attn_decode(flux_ctx* c, const uint16_t* q, const uint16_t* k_cache,
+                     const uint16_t* v_cache, int S_max, const int32_t* seqlens, uint16_t* o,
+                     float* lse, int B, int Hq, int Hkv, int d, const uint8_t* layer_mode,
+                     int layer, int sink_blocks, int window_blocks, int block, float scale,
+                     flux_stream_t stream) {
+  if (!c || !q || !k_cache || !v_cache || !seqlens || !o)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: null tensor");
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode: sizes must be positive");
+  if (d != 64 && d != 128)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode: head_dim %d (supported: 64, 128)", d);
+  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode: Hq/Hkv must be 1, 2 or 4 (%d, %d)", Hq,
+                Hkv);
+  if (block < 1 || sink_blocks < 0 || window_blocks < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: bad block / sink / window");
+  if (layer_mode && layer < 0) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: negative layer");
+  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: scale must be finite and positive");
+  if (static_cast<long long>(B) * Hkv > kMaxTickets)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode: B * Hkv > %d", kMaxTickets);
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: tensors must be 16-byte aligned");
+  flux::DecodeLaunch p;
+  flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
+                    &p.chunk_fa, &p.chunk_sa);
+  const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
+  const size_t o_bytes = align256(rows * d * sizeof(float));
+  const size_t need = o_bytes + align256(rows * 2 * sizeof(float));
+  if (need > c->workspace_bytes)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode: workspace %zu < %zu bytes", c->workspace_bytes,
+                need);
+  CUtensorMap tk, tv;
+  int rc;
+  if ((rc = make_map_4d(&tk, k_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, v_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.S_max = S_max;
+  p.q = q;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.layer_mode = layer_mode;
+  p.layer = layer;
+  p.sink_blocks = sink_blocks;
+  p.window_blocks = window_blocks;
+  p.block = block;
+  p.scale = scale;
+  p.part_o = static_cast<float*>(c->workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
+  p.tickets = c->tickets;
+  p.st = status_of(c);
+  const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode: launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// kernels.h -- internal launcher interfaces between the C ABI (api.cu) and
+// the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace flux {
+
+struct PrefillLaunch {
+  int B, T, Hq, Hkv, d;
+  int block, nqb;
+  float scale;
+  const uint8_t* layer_mode;
+  int layer;
+  const int32_t* row_ptr;
+  const int32_t* col;
+  uint16_t* o;
+  float* lse;
+  DevStatus st;
+};
+int prefill_smem_bytes(int d);
+cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const PrefillLaunch& p, cudaStream_t stream);
+
+struct DecodeLaunch {
+  int B, Hq, Hkv, d, S_max;
+  const uint16_t* q;
+  const int32_t* seqlens;
+  uint16_t* o;
+  float* lse;
+  const uint8_t* layer_mode;
+  int layer;
+  int sink_blocks, window_blocks, block;
+  float scale;
+  int nsplit, chunk_fa, chunk_sa;
+  float* part_o;    // [B, Hq, nsplit, d]
+  float* part_ml;   // [B, Hq, nsplit, 2]
+  int* tickets;     // [B, Hkv], zero between calls
+  DevStatus st;
+};
+// Split plan for a shape (host only): number of splits and chunk lengths.
+void decode_plan(int B, int Hkv, int S_max, int sink_blocks, int window_blocks, int block,
+                 int num_sms, int* nsplit, int* chunk_fa, int* chunk_sa);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int nsplit);
+cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeLaunch& p,
+                          cudaStream_t stream);
+
+struct RouteLaunch {
+  const uint16_t* hidden;
+  int T, Hd, n_pool;
+  const float* W1;
+  const float* b1;
+  int H1;
+  const float* W2;
+  const float* b2;
+  int L;
+  float thresh;
+  uint8_t* layer_mode;
+  float* score;
+  float* pooled;   // workspace [2 Hd]
+  float* hidden1;  // workspace [H1]
+  int* ticket;     // workspace, zero between calls
+};
+size_t route_workspace_bytes(int Hd, int H1);
+cudaError_t launch_route(const RouteLaunch& p, cudaStream_t stream);
+
+cudaError_t launch_streaming_mask(int nqb, int nkb, int sink, int window, uint8_t* mask,
+                                  cudaStream_t stream);
+cudaError_t launch_block_index(const uint8_t* mask, int nqb, int nkb, int32_t* row_ptr,
+                               int32_t* col, int cap, int32_t* counts, int* err,
+                               cudaStream_t stream);
+
+}  // namespace flux

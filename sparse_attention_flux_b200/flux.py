@@ -1,0 +1,242 @@
+"""Thin Python binding of libflux (the C ABI in include/flux.h).
+
+Argument marshalling only: every step of the routed-attention path runs in
+the CUDA kernels of libflux.so.  Tensors are torch tensors on the CUDA device
+(torch provides device memory and streams); their data pointers and the
+current torch stream are passed straight through the C ABI.  There is no CPU
+fallback: if libflux.so is missing or a call fails, an exception is raised.
+
+Names follow the C ABI: ``route``, ``build_streaming_mask``,
+``build_block_index``, ``attn_prefill``, ``attn_decode``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libflux.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "flux.h")
+
+FLUX_OK = 0
+FLUX_ERR_INVALID_ARG = -1
+FLUX_ERR_SHAPE = -2
+FLUX_ERR_UNSUPPORTED = -3
+FLUX_ERR_CUDA = -4
+FLUX_ERR_TIMEOUT = -5
+FLUX_ERR_DEVICE_CHECK = -6
+
+
+class FluxError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libflux error {code}: {msg}")
+        self.code = code
+
+
+_lock = threading.Lock()
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+_SIGNATURES = {
+    "flux_version": ([], _i),
+    "flux_last_error": ([], ctypes.c_char_p),
+    "flux_ctx_create": ([ctypes.POINTER(_vp), _i, ctypes.c_size_t], _i),
+    "flux_ctx_destroy": ([_vp], _i),
+    "flux_ctx_check": ([_vp, _vp], _i),
+    "flux_ctx_set_spin_limit_ms": ([_vp, _i], _i),
+    "flux_route": ([_vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _i, _f, _vp, _vp, _vp], _i),
+    "flux_build_streaming_mask": ([_i, _i, _i, _i, _vp, _vp], _i),
+    "flux_build_block_index": ([_vp, _vp, _i, _i, _vp, _vp, _i, _vp], _i),
+    "flux_attn_prefill": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
+                           _i, _i, _f, _vp], _i),
+    "flux_attn_decode": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i, _i, _i,
+                          _i, _f, _vp], _i),
+    "flux_decode_workspace_bytes": ([_vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                                     ctypes.POINTER(ctypes.c_size_t)], _i),
+}
+
+
+def header_symbols(path: str = HEADER):
+    """Function names declared in include/flux.h."""
+    with open(path) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(flux_\w+)\s*\(", text, flags=re.M)))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libflux.so (built in-tree by sparse_attention_flux_b200.build)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m sparse_attention_flux_b200.build`"
+                    " (there is no CPU fallback)")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (args, res) in _SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != FLUX_OK:
+        raise FluxError(rc, lib().flux_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, name, device=None):
+    import torch
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+class Context:
+    """Owns a flux_ctx: the device workspace and the device error word."""
+
+    def __init__(self, device: int = 0, workspace_bytes: int = 0):
+        import torch
+        self.device = torch.device("cuda", device)
+        h = ctypes.c_void_p()
+        _check(lib().flux_ctx_create(ctypes.byref(h), device, workspace_bytes))
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().flux_ctx_destroy(self._h)
+            self._h = None
+
+    def __del__(self):  # pragma: no cover - interpreter shutdown order
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    @property
+    def handle(self):
+        return self._h
+
+    def check(self, stream=None) -> None:
+        """Synchronize the stream and raise if a device-side check failed."""
+        _check(lib().flux_ctx_check(self._h, _stream(stream)))
+
+    def set_spin_limit_ms(self, ms: int) -> None:
+        _check(lib().flux_ctx_set_spin_limit_ms(self._h, int(ms)))
+
+    def decode_workspace_bytes(self, B, Hq, Hkv, d, S_max, sink_blocks, window_blocks, block) -> int:
+        n = ctypes.c_size_t()
+        _check(lib().flux_decode_workspace_bytes(self._h, B, Hq, Hkv, d, S_max, sink_blocks,
+                                                 window_blocks, block, ctypes.byref(n)))
+        return n.value
+
+    # ------------------------------------------------------------------ router
+    def route(self, hidden, W1, b1, W2, b2, thresh: float, layer_mode, score=None,
+              n_pool: int = 100, stream=None):
+        import torch
+        _need(hidden, torch.bfloat16, "hidden", self.device)
+        for n_, t in (("W1", W1), ("b1", b1), ("W2", W2), ("b2", b2), ("score", score)):
+            _need(t, torch.float32, n_, self.device)
+        _need(layer_mode, torch.uint8, "layer_mode", self.device)
+        T, Hd = hidden.shape
+        H1, L = W1.shape[0], W2.shape[0]
+        if W1.shape != (H1, 2 * Hd) or W2.shape != (L, H1) or b1.numel() != H1 or b2.numel() != L:
+            raise ValueError("router weight shapes do not match hidden")
+        if layer_mode.numel() < L or (score is not None and score.numel() < L):
+            raise ValueError("layer_mode/score too small")
+        _check(lib().flux_route(self._h, _ptr(hidden), T, Hd, n_pool, _ptr(W1), _ptr(b1), H1,
+                                _ptr(W2), _ptr(b2), L, float(thresh), _ptr(layer_mode),
+                                _ptr(score), _stream(stream)))
+
+    # ------------------------------------------------------------------ masks
+    def build_streaming_mask(self, nqb: int, nkb: int, sink_blocks: int, window_blocks: int,
+                             block_mask, stream=None):
+        import torch
+        _need(block_mask, torch.uint8, "block_mask", self.device)
+        if block_mask.numel() < nqb * nkb:
+            raise ValueError("block_mask too small")
+        _check(lib().flux_build_streaming_mask(nqb, nkb, sink_blocks, window_blocks,
+                                               _ptr(block_mask), _stream(stream)))
+
+    def build_block_index(self, block_mask, row_ptr, col, stream=None):
+        import torch
+        _need(block_mask, torch.uint8, "block_mask", self.device)
+        _need(row_ptr, torch.int32, "row_ptr", self.device)
+        _need(col, torch.int32, "col", self.device)
+        nqb, nkb = block_mask.shape
+        if row_ptr.numel() < nqb + 1:
+            raise ValueError("row_ptr needs nqb + 1 entries")
+        _check(lib().flux_build_block_index(self._h, _ptr(block_mask), nqb, nkb, _ptr(row_ptr),
+                                            _ptr(col), col.numel(), _stream(stream)))
+
+    # ------------------------------------------------------------------ attention
+    def attn_prefill(self, q, k, v, o, scale: float, layer_mode=None, layer: int = 0,
+                     row_ptr=None, col=None, block: int = 128, lse=None, stream=None):
+        import torch
+        for n_, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+            _need(t, torch.bfloat16, n_, self.device)
+        _need(lse, torch.float32, "lse", self.device)
+        _need(layer_mode, torch.uint8, "layer_mode", self.device)
+        _need(row_ptr, torch.int32, "row_ptr", self.device)
+        _need(col, torch.int32, "col", self.device)
+        B, T, Hq, d = q.shape
+        Hkv = k.shape[2]
+        if k.shape != (B, T, Hkv, d) or v.shape != k.shape or o.shape != q.shape:
+            raise ValueError("q/k/v/o shapes are inconsistent")
+        if lse is not None and lse.numel() < B * Hq * T:
+            raise ValueError("lse too small")
+        nqb = 0 if row_ptr is None else row_ptr.numel() - 1
+        _check(lib().flux_attn_prefill(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
+                                       T, Hq, Hkv, d, _ptr(layer_mode), layer, _ptr(row_ptr),
+                                       _ptr(col), nqb, block, float(scale), _stream(stream)))
+
+    def attn_decode(self, q, k_cache, v_cache, seqlens, o, scale: float, layer_mode=None,
+                    layer: int = 0, sink_blocks: int = 1, window_blocks: int = 16,
+                    block: int = 128, lse=None, stream=None):
+        import torch
+        for n_, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("o", o)):
+            _need(t, torch.bfloat16, n_, self.device)
+        _need(seqlens, torch.int32, "seqlens", self.device)
+        _need(lse, torch.float32, "lse", self.device)
+        _need(layer_mode, torch.uint8, "layer_mode", self.device)
+        B, Hq, d = q.shape
+        _, S_max, Hkv, _ = k_cache.shape
+        if k_cache.shape != (B, S_max, Hkv, d) or v_cache.shape != k_cache.shape:
+            raise ValueError("cache shapes are inconsistent")
+        if o.shape != q.shape or seqlens.numel() < B:
+            raise ValueError("o/seqlens shapes are inconsistent")
+        if lse is not None and lse.numel() < B * Hq:
+            raise ValueError("lse too small")
+        _check(lib().flux_attn_decode(self._h, _ptr(q), _ptr(k_cache), _ptr(v_cache), S_max,
+                                      _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, d,
+                                      _ptr(layer_mode), layer, sink_blocks, window_blocks, block,
+                                      float(scale), _stream(stream)))

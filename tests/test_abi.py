@@ -1,0 +1,59 @@
+"""The C-ABI library: it loads, exports every symbol include/flux.h declares,
+and rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+
+import pytest
+
+from sparse_attention_flux_b200 import build, flux
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build(quiet=True)
+    return flux.lib()
+
+
+def test_header_declares_the_hot_path_entry_points():
+    names = flux.header_symbols()
+    for must in ("flux_route", "flux_build_streaming_mask", "flux_build_block_index",
+                 "flux_attn_prefill", "flux_attn_decode", "flux_ctx_create", "flux_ctx_destroy",
+                 "flux_ctx_check", "flux_last_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in flux.header_symbols():
+        assert hasattr(lib, name), f"libflux.so does not export {name}"
+
+
+def test_binding_covers_every_declared_symbol():
+    assert set(flux.header_symbols()) <= set(flux._SIGNATURES)
+
+
+def test_library_is_built_for_sm100a_and_in_tree(lib):
+    assert os.path.dirname(flux.LIB_PATH) == os.path.dirname(os.path.abspath(flux.__file__))
+    assert lib.flux_version() == 1
+
+
+def test_host_side_argument_checks_need_no_gpu(lib):
+    # Null pointers and bad sizes are rejected before any CUDA call.
+    assert lib.flux_build_streaming_mask(4, 4, 1, 2, None, None) == flux.FLUX_ERR_INVALID_ARG
+    assert b"null" in lib.flux_last_error()
+    assert lib.flux_build_streaming_mask(4, 4, 1, 0, ctypes.c_void_p(16), None) == \
+        flux.FLUX_ERR_INVALID_ARG
+    assert lib.flux_route(None, None, 1, 1, 1, None, None, 1, None, None, 1, 0.5, None, None,
+                          None) == flux.FLUX_ERR_INVALID_ARG
+    assert lib.flux_attn_prefill(None, None, None, None, None, None, 1, 1, 1, 1, 128, None, 0,
+                                 None, None, 0, 128, 0.1, None) == flux.FLUX_ERR_INVALID_ARG
+    assert lib.flux_attn_decode(None, None, None, None, 1, None, None, None, 1, 1, 1, 128, None,
+                                0, 1, 1, 128, 0.1, None) == flux.FLUX_ERR_INVALID_ARG
+    assert lib.flux_ctx_destroy(None) == flux.FLUX_ERR_INVALID_ARG
+    assert lib.flux_ctx_check(None, None) == flux.FLUX_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(flux, "LIB_PATH", str(tmp_path / "libflux.so"))
+    monkeypatch.setattr(flux, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        flux.lib()
