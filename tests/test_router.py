@@ -56,7 +56,9 @@ def test_route_qwen3_4b_router_workload(ctx):
     assert np.array_equal(mode_g, mode_o)
     np.testing.assert_allclose(score_g, r, rtol=0, atol=2e-6)
     assert 8 <= int(mode_o.sum()) <= 28       # about half the layers go to each mode
-    assert np.abs(z).min() > 0.25              # the margin the workload is built with
+    # The +-2 coin biases keep every logit far from the threshold's fp32 rounding gap
+    # (|z| ~ 1e-6 would be needed for fp32 and fp64 to disagree).
+    assert np.abs(z).min() > 0.05, np.abs(z).min()
 
 
 def test_route_threshold_and_tie(ctx):
