@@ -174,6 +174,38 @@ int flux_attn_decode(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_cache,
                      int sink_blocks, int window_blocks, int block, float scale,
                      flux_stream_t stream);
 
+/* --------------------------------------------------------------------------
+ * Decode attention that allocates nothing.  The pages have no counterpart of
+ * this entry point; it exists for callers that cannot call cudaMalloc: an
+ * inference engine that reserves all device memory up front and owns every
+ * later allocation through its own pool, a plugin host that forbids libraries
+ * from allocating, or a latency-critical loop that cannot afford cudaMalloc's
+ * implicit device synchronisation.  Such callers cannot create a flux_ctx, so
+ * this variant of flux_attn_decode keeps its split-KV scratch (partials,
+ * merge tickets, error word) in one file-scope static device array of
+ * 32 MiB inside libflux.so, which every GPU that loads the library holds until
+ * the process exits.
+ *   Arguments, layouts and results are those of flux_attn_decode, without the
+ *   ctx.  status: optional device int32 that receives the device error word
+ *   of this call (0 = OK, 2 = a seqlens entry out of range, 1 = a bounded
+ *   wait ran out); NULL to skip.
+ *   Limits: B * Hkv <= 4096 and B * Hq * nsplit * (d + 2) * 4 bytes of
+ *   partials within the 32 MiB (nsplit as flux_decode_workspace_bytes plans
+ *   it; e.g. B 16, Hq 32, d 128 at 131072 tokens needs 17 MiB).  Larger shapes
+ *   return FLUX_ERR_SHAPE before any device work.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  Every call clears the error word and the
+ *   tickets it uses on `stream`, then reuses the same array: calls that
+ *   overlap on the GPU (on different streams or host threads) race and must
+ *   be serialised by the caller. */
+int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
+                             int S_max, const int32_t* seqlens, uint16_t* o, float* lse,
+                             int B, int Hq, int Hkv, int d,
+                             const uint8_t* layer_mode, int layer,
+                             int sink_blocks, int window_blocks, int block, float scale,
+                             int32_t* status, flux_stream_t stream);
+
 /* Workspace bytes flux_attn_decode needs on this ctx's device for this shape
  * and SA window (host-only query; no device work). */
 int flux_decode_workspace_bytes(flux_ctx* ctx, int B, int Hq, int Hkv, int d, int S_max,

@@ -361,3 +361,135 @@ int flux_attn_decode(flux_ctx* c, const uint16_t* q, const uint16_t* k_cache,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// flux_attn_decode_noalloc: flux_attn_decode for callers that cannot call
+// cudaMalloc (an engine that owns all device memory through its own pool, a
+// plugin host that forbids library allocations, a loop that cannot take
+// cudaMalloc's implicit synchronisation).  Its scratch is the static array
+// below, which every device that loads libflux.so holds until the process
+// exits.  Host code must not pass the array's name to a kernel -- on the host
+// it is only a stand-in symbol -- so each device's address is looked up once,
+// with that device current, and cached.
+namespace {
+
+constexpr size_t kNoAllocBytes = size_t(32) << 20;        // 32 MiB
+constexpr int kNoAllocMaxGroups = 4096;                    // B * Hkv
+constexpr size_t kNoAllocErrOff = 0;                       // error word
+constexpr size_t kNoAllocTicketOff = 256;                  // [kNoAllocMaxGroups] int
+constexpr size_t kNoAllocPartOff = kNoAllocTicketOff + kNoAllocMaxGroups * sizeof(int);
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+struct NoAllocDevice {
+  bool ready;
+  char* base;   // device address of g_noalloc_scratch on this device
+  int num_sms;
+};
+constexpr int kNoAllocMaxDevices = 64;
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+std::mutex g_noalloc_mu;
+
+int noalloc_setup(NoAllocDevice** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_noalloc: device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& d = g_noalloc_dev[dev];
+  if (!d.ready) {
+    void* ptr = nullptr;
+    if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess)
+      return cuda_fail(e, "flux_attn_decode_noalloc: cudaGetSymbolAddress");
+    int sms = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "flux_attn_decode_noalloc: SM count");
+    d.base = static_cast<char*>(ptr);
+    d.num_sms = sms;
+    d.ready = true;
+  }
+  *out = &d;
+  return FLUX_OK;
+}
+
+}  // namespace
+
+extern "C" int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cache,
+                                        const uint16_t* v_cache, int S_max,
+                                        const int32_t* seqlens, uint16_t* o, float* lse, int B,
+                                        int Hq, int Hkv, int d, const uint8_t* layer_mode,
+                                        int layer, int sink_blocks, int window_blocks, int block,
+                                        float scale, int32_t* status, flux_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !seqlens || !o)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: null tensor");
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_noalloc: sizes must be positive");
+  if (d != 64 && d != 128)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_noalloc: head_dim %d (supported: 64, 128)",
+                d);
+  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_noalloc: Hq/Hkv must be 1, 2 or 4");
+  if (block < 1 || sink_blocks < 0 || window_blocks < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: bad block / sink / window");
+  if (layer_mode && layer < 0)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: negative layer");
+  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: scale must be finite and positive");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: tensors must be 16-byte aligned");
+  if (static_cast<long long>(B) * Hkv > kNoAllocMaxGroups)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_noalloc: B * Hkv = %lld exceeds %d",
+                static_cast<long long>(B) * Hkv, kNoAllocMaxGroups);
+  NoAllocDevice* dev = nullptr;
+  int rc = noalloc_setup(&dev);
+  if (rc != FLUX_OK) return rc;
+  flux::DecodeLaunch p;
+  flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, dev->num_sms, &p.nsplit,
+                    &p.chunk_fa, &p.chunk_sa);
+  const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
+  const size_t ml_bytes = align256(rows * 2 * sizeof(float));
+  const size_t o_bytes = align256(rows * d * sizeof(float));
+  if (kNoAllocPartOff + ml_bytes + o_bytes > kNoAllocBytes)
+    return fail(FLUX_ERR_SHAPE,
+                "flux_attn_decode_noalloc: %zu bytes of split partials exceed the %zu-byte static "
+                "scratch (use flux_attn_decode with a ctx for this shape)",
+                ml_bytes + o_bytes, kNoAllocBytes - kNoAllocPartOff);
+  CUtensorMap tk, tv;
+  if ((rc = make_map_4d(&tk, k_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, v_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = reinterpret_cast<int*>(dev->base + kNoAllocErrOff);
+  int* tickets = reinterpret_cast<int*>(dev->base + kNoAllocTicketOff);
+  // The array keeps the previous call's contents: the error word and this
+  // call's tickets must start at zero.
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(tickets, 0, static_cast<size_t>(B) * Hkv * sizeof(int), s);
+  if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: clear scratch");
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.S_max = S_max;
+  p.q = q;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.layer_mode = layer_mode;
+  p.layer = layer;
+  p.sink_blocks = sink_blocks;
+  p.window_blocks = window_blocks;
+  p.block = block;
+  p.scale = scale;
+  p.part_ml = reinterpret_cast<float*>(dev->base + kNoAllocPartOff);
+  p.part_o = reinterpret_cast<float*>(dev->base + kNoAllocPartOff + ml_bytes);
+  p.tickets = tickets;
+  p.st = flux::DevStatus{err, 2000LL * 1000000LL};
+  e = flux::launch_decode(tk, tv, p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: launch");
+  if (status && (e = cudaMemcpyAsync(status, err, sizeof(int), cudaMemcpyDeviceToDevice, s)) !=
+                    cudaSuccess)
+    return cuda_fail(e, "flux_attn_decode_noalloc: copy status");
+  return FLUX_OK;
+}

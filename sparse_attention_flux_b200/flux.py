@@ -58,6 +58,8 @@ _SIGNATURES = {
                           _i, _f, _vp], _i),
     "flux_decode_workspace_bytes": ([_vp, _i, _i, _i, _i, _i, _i, _i, _i,
                                      ctypes.POINTER(ctypes.c_size_t)], _i),
+    "flux_attn_decode_noalloc": ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i, _i,
+                                  _i, _i, _f, _vp, _vp], _i),
 }
 
 
@@ -240,3 +242,25 @@ class Context:
                                       _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, d,
                                       _ptr(layer_mode), layer, sink_blocks, window_blocks, block,
                                       float(scale), _stream(stream)))
+
+
+def attn_decode_noalloc(q, k_cache, v_cache, seqlens, o, scale: float, layer_mode=None,
+                        layer: int = 0, sink_blocks: int = 1, window_blocks: int = 16,
+                        block: int = 128, lse=None, status=None, stream=None):
+    """flux_attn_decode_noalloc: decode without a Context; scratch lives in a static
+    32 MiB device array inside libflux.so (see include/flux.h for the limits)."""
+    import torch
+    for n_, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("o", o)):
+        _need(t, torch.bfloat16, n_)
+    _need(seqlens, torch.int32, "seqlens")
+    _need(lse, torch.float32, "lse")
+    _need(layer_mode, torch.uint8, "layer_mode")
+    _need(status, torch.int32, "status")
+    B, Hq, d = q.shape
+    _, S_max, Hkv, _ = k_cache.shape
+    if k_cache.shape != (B, S_max, Hkv, d) or v_cache.shape != k_cache.shape or o.shape != q.shape:
+        raise ValueError("q/cache/o shapes are inconsistent")
+    _check(lib().flux_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), S_max,
+                                          _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, d,
+                                          _ptr(layer_mode), layer, sink_blocks, window_blocks,
+                                          block, float(scale), _ptr(status), _stream(stream)))
