@@ -138,7 +138,8 @@ int flux_build_block_index(flux_ctx* ctx, const uint8_t* block_mask, int nqb, in
  *   the CSR list).  layer_mode == NULL means FA.
  *   row_ptr/col: the CSR list from flux_build_block_index over nqb >=
  *   ceil(T / block) q-blocks; required unless layer_mode == NULL.
- *   block: 64 or a multiple of 128.  d: 64 or 128.  scale: score scale
+ *   block: 64 or a multiple of 128.  d: 64 or 128.  With layer_mode given,
+ *   T <= 262144 (the CTA's key-tile list lives in shared memory).  scale: score scale
  *   (1/sqrt(d) for the models on the pages).
  * Runs the tcgen05/TMEM/TMA flash-attention kernel; skipped blocks are never
  * loaded.  Errors: UNSUPPORTED for other d or block, or Hq % Hkv != 0; SHAPE

@@ -262,6 +262,9 @@ int flux_attn_prefill(flux_ctx* c, const uint16_t* q, const uint16_t* k, const u
     if (nqb < (T + block - 1) / block)
       return fail(FLUX_ERR_SHAPE, "flux_attn_prefill: nqb %d < ceil(T / block) = %d", nqb,
                   (T + block - 1) / block);
+    if ((T + 127) / 128 > flux::kPrefillMaxKvTiles)
+      return fail(FLUX_ERR_SHAPE, "flux_attn_prefill: routed prefill supports T <= %d",
+                  flux::kPrefillMaxKvTiles * 128);
   }
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: tensors must be 16-byte aligned");

@@ -11,6 +11,10 @@
 
 namespace flux {
 
+// A routed (block-index) prefill keeps its key-tile list in shared memory:
+// at most this many 128-column key tiles, i.e. T <= 262144.
+constexpr int kPrefillMaxKvTiles = 2048;
+
 struct PrefillLaunch {
   int B, T, Hq, Hkv, d;
   int block, nqb;

@@ -3,20 +3,28 @@
 // Flux Attention routes each layer to Full Attention (exact causal softmax
 // attention) or to block-sparse Sparse Attention (arXiv abstract; model card
 // "Flux Attention: Qwen3-4B", "Sample Usage").  One kernel serves both: a
-// CTA owns one 128-row query tile of one (batch, query head) and walks a list
-// of 128-column key tiles -- every tile up to the diagonal for FA, the tiles
-// named by the compressed block-index list for SA -- so skipped blocks are
-// never loaded.
+// CTA owns 256 query rows -- two 128-row tiles Q0, Q1 -- of one (batch, query
+// head) and walks a list of 128-column key tiles: every tile up to the
+// diagonal for FA, the tiles named by the compressed block-index list for SA
+// (built once per CTA into shared memory), so skipped blocks are never loaded.
+// Each K/V tile is loaded once and used by both query tiles.
 //
-// Per CTA (192 threads, warp-specialised):
-//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring.
-//   warp 1      TMEM owner and UMMA issuer: S = Q K^T into TMEM (fp32), then
-//               O += P V into TMEM, tcgen05.commit onto mbarriers.
-//   warps 2..5  softmax: one query row per thread (= one TMEM lane), online
-//               softmax in the log2 domain, P written to shared memory as
-//               bf16 in the 128-byte-swizzled K-major layout UMMA reads,
-//               lazy O rescale, and the epilogue O / l -> bf16.
-// The S MMA of tile j+1 overlaps the exponentials of tile j.
+// Per CTA (384 threads, warp-specialised):
+//   warp 0      TMA producer (Q0, Q1 once; K/V tiles into a 2-stage ring) and,
+//               for SA, the builder of the CTA's key-tile list.
+//   warp 1      TMEM owner (all 512 columns) and UMMA issuer:
+//                 S_i = Q_i K^T             (A, B from shared memory)
+//                 O_i += P_i V              (A = P_i from TMEM, B from smem)
+//               issued in the order S0 S1 | PV0 S0' PV1 S1' | ... so that the
+//               tensor core works on one tile while the other's softmax runs.
+//   warps 2, 3  idle.
+//   warps 4-7   softmax of Q0, warps 8-11 softmax of Q1: one query row per
+//               thread (= one TMEM lane); online softmax in the log2 domain;
+//               P_i written back over S_i's columns as packed bf16 for the
+//               TMEM-A MMA; O_i rescaled only when the row max grows by more
+//               than 2^8 (exact: the final division uses the same max); the
+//               epilogue writes O_i / l.
+// TMEM columns: S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [384,384+D).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,14 +32,16 @@ namespace flux {
 
 namespace {
 
-constexpr int kBM = 128;            // query rows per CTA (TMEM lanes)
-constexpr int kBN = 128;            // key columns per tile
-constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one swizzle-128B box)
-constexpr int kThreads = 192;
+constexpr int kBM = 128;                  // query rows per tile (TMEM lanes)
+constexpr int kBN = 128;                  // key columns per tile
+constexpr int kChunkBytes = 128 * 128;    // 128 rows x 64 bf16: one swizzle-128B box
+constexpr int kThreads = 384;
+constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold, log2 units
 
 struct PrefillArgs {
   int B, T, Hq, Hkv, G;
-  int nqt;           // number of 128-row tiles along T
+  int npair;         // 256-row query pairs along T
+  int nkt;           // 128-column key tiles along T
   int block;         // mask block: 64 or a multiple of 128
   int nqb;           // rows of the CSR
   int nkb;           // kv blocks along T (valid CSR column range)
@@ -45,127 +55,74 @@ struct PrefillArgs {
   DevStatus st;
 };
 
-// The sequence of key tiles a query tile visits, identical in every role.
-// sub-mask bit (r * 2 + c): query half r (rows 64r..64r+63) may see key half
-// c (columns 64c..64c+63); only a 64-token mask block makes it partial.
-struct TileIter {
-  int fa, I, m;      // m = block / 128 (>= 1), or 0 for block == 64
-  int J;             // FA cursor
-  int p0, e0, p1, e1, sub;
-  const int32_t* col;
-  int nkb;
-  int* err;
-
-  __device__ void init(const PrefillArgs& a, int qt, bool is_fa) {
-    fa = is_fa;
-    I = qt;
-    J = 0;
-    sub = 0;
-    col = a.col;
-    nkb = a.nkb;
-    err = a.st.err;
-    p0 = e0 = p1 = e1 = 0;
-    m = a.block >= 128 ? a.block / 128 : 0;
-    if (fa) return;
-    const int nnz = a.row_ptr[a.nqb];
-    auto row = [&](int qb, int& p, int& e) {
-      p = e = 0;
-      if (qb >= a.nqb) return;
-      int lo = a.row_ptr[qb], hi = a.row_ptr[qb + 1];
-      if (lo < 0 || hi < lo || hi > nnz) {
-        raise_error(err, DEV_ERR_CSR);
-        return;
-      }
-      p = lo;
-      e = hi;
-    };
-    if (m >= 1) {
-      row(qt / m, p0, e0);
-    } else {
-      row(2 * qt, p0, e0);
-      row(2 * qt + 1, p1, e1);
-    }
-  }
-
-  __device__ int entry(int p) {
-    int j = col[p];
-    if (j < 0 || j >= nkb) {
-      raise_error(err, DEV_ERR_CSR);
-      return -1;
-    }
-    return j;
-  }
-
-  __device__ bool next(int& Jo, uint32_t& sm) {
-    if (fa) {
-      if (J > I) return false;
-      Jo = J++;
-      sm = 0xFu;
-      return true;
-    }
-    if (m >= 1) {
-      while (p0 < e0) {
-        int j = entry(p0);
-        if (j < 0) { ++p0; sub = 0; continue; }
-        int t = j * m + sub;
-        if (t > I) { p0 = e0; return false; }   // ascending list: nothing further is causal
-        if (++sub == m) { sub = 0; ++p0; }
-        Jo = t;
-        sm = 0xFu;
-        return true;
-      }
-      return false;
-    }
-    // block == 64: merge the lists of query blocks 2I and 2I+1 by key tile j/2.
-    for (;;) {
-      int j0 = -1, j1 = -1;
-      while (p0 < e0 && (j0 = entry(p0)) < 0) ++p0;
-      while (p1 < e1 && (j1 = entry(p1)) < 0) ++p1;
-      if (p0 >= e0) j0 = -1;
-      if (p1 >= e1) j1 = -1;
-      if (j0 < 0 && j1 < 0) return false;
-      int t0 = j0 >= 0 ? (j0 >> 1) : 0x7fffffff;
-      int t1 = j1 >= 0 ? (j1 >> 1) : 0x7fffffff;
-      int t = t0 < t1 ? t0 : t1;
-      if (t > I) { p0 = e0; p1 = e1; return false; }
-      uint32_t bits = 0;
-      while (p0 < e0) {
-        int j = entry(p0);
-        if (j >= 0 && (j >> 1) != t) break;
-        if (j >= 0) bits |= 1u << (0 * 2 + (j & 1));
-        ++p0;
-      }
-      while (p1 < e1) {
-        int j = entry(p1);
-        if (j >= 0 && (j >> 1) != t) break;
-        if (j >= 0) bits |= 1u << (1 * 2 + (j & 1));
-        ++p1;
-      }
-      if (bits == 0) continue;
-      Jo = t;
-      sm = bits;
-      return true;
-    }
-  }
-};
-
-// Bars: 0 q_full | 1,2 k_full | 3,4 v_full | 5,6 kv_empty | 7 s_full | 8 s_free
-//       9 p_full | 10 o_done | 11 drain
-enum { B_Q = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_SFREE = 8, B_PF = 9, B_OD = 10,
-       B_DRAIN = 11, B_COUNT = 12 };
+enum { B_Q = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_PF = 9, B_OD = 11, B_DRAIN = 12,
+       B_COUNT = 13 };
 
 template <int D>
 struct Smem {
   static constexpr int CH = D / 64;
-  static constexpr int Q = 0;
-  static constexpr int K = Q + CH * kChunkBytes;
-  static constexpr int V = K + 2 * CH * kChunkBytes;
-  static constexpr int P = V + 2 * CH * kChunkBytes;
-  static constexpr int BARS = P + 2 * kChunkBytes;
+  static constexpr int Q = 0;                                  // [2 tiles][CH chunks]
+  static constexpr int K = Q + 2 * CH * kChunkBytes;           // [2 stages][CH]
+  static constexpr int V = K + 2 * CH * kChunkBytes;           // [2 stages][CH]
+  static constexpr int MAP = V + 2 * CH * kChunkBytes;         // u32 [kPrefillMaxKvTiles]
+  static constexpr int LIST = MAP + 4 * kPrefillMaxKvTiles;    // u32 [kPrefillMaxKvTiles]
+  static constexpr int BARS = LIST + 4 * kPrefillMaxKvTiles;
   static constexpr int TMEM_SLOT = BARS + B_COUNT * 8;
-  static constexpr int TOTAL = TMEM_SLOT + 16;
+  static constexpr int NLIST = TMEM_SLOT + 4;
+  static constexpr int TOTAL = NLIST + 12;
   static constexpr int ALLOC = TOTAL + 1024;  // room to align the base to 1024
 };
+
+// SA: the CTA's key tiles and, per tile, which (64-row query sub-block,
+// 64-column key sub-block) pairs the block mask keeps: bit (qs * 2 + ks).
+// One warp: OR every kept block of the (up to four) CSR rows the CTA's query
+// rows fall in into a per-tile map, then compact it in ascending tile order.
+// Returns the list length.  Tiles past the last query row's diagonal are
+// dropped (causal), CSR entries out of range raise DEV_ERR_CSR and are skipped.
+__device__ int build_tile_list(const PrefillArgs& a, int pair, uint32_t* map, uint32_t* list) {
+  const int lane = threadIdx.x & 31;
+  const int last = min(2 * pair + 1, a.nkt - 1);
+  for (int J = lane; J <= last; J += 32) map[J] = 0;
+  __syncwarp();
+  const int nnz = a.row_ptr[a.nqb];
+  for (int qs = 0; qs < 4; ++qs) {
+    const int row = pair * 256 + qs * 64;
+    if (row >= a.T) break;
+    const int qb = row / a.block;
+    if (qb >= a.nqb) {
+      if (lane == 0) raise_error(a.st.err, DEV_ERR_CSR);
+      break;
+    }
+    int lo = a.row_ptr[qb], hi = a.row_ptr[qb + 1];
+    if (lo < 0 || hi < lo || hi > nnz) {
+      if (lane == 0) raise_error(a.st.err, DEV_ERR_CSR);
+      continue;
+    }
+    for (int e = lo + lane; e < hi; e += 32) {
+      const int j = a.col[e];
+      if (j < 0 || j >= a.nkb) {
+        raise_error(a.st.err, DEV_ERR_CSR);
+        continue;
+      }
+      const int k0 = j * a.block, k1 = min((j + 1) * a.block, a.T);   // key range of block j
+      for (int ks = k0 >> 6; ks < (k1 + 63) >> 6; ++ks) {                 // 64-column sub-blocks
+        const int J = ks >> 1;
+        if (J > last) break;
+        atomicOr(&map[J], 1u << (qs * 2 + (ks & 1)));
+      }
+    }
+  }
+  __syncwarp();
+  int n = 0;
+  for (int base = 0; base <= last; base += 32) {
+    const int J = base + lane;
+    const uint32_t m = J <= last ? map[J] : 0u;
+    const unsigned bal = __ballot_sync(0xffffffffu, m != 0);
+    if (m != 0) list[n + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint32_t>(J) | (m << 24);
+    n += __popc(bal);
+  }
+  return n;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -174,33 +131,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
   using L = Smem<D>;
   constexpr int CH = L::CH;
-  constexpr uint32_t kTmemCols = 256;  // S: 128 columns, O: D columns
+  constexpr uint32_t kTmemCols = 512;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem + L::Q;
   uint8_t* sK = smem + L::K;
   uint8_t* sV = smem + L::V;
-  uint8_t* sP = smem + L::P;
+  uint32_t* map = reinterpret_cast<uint32_t*>(smem + L::MAP);
+  uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::LIST);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BARS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::TMEM_SLOT);
+  int* nlist = reinterpret_cast<int*>(smem + L::NLIST);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Longest-first order: the last query tiles carry the most causal work.
-  const int per_tile = a.Hq * a.B;
-  const int qt = a.nqt - 1 - static_cast<int>(blockIdx.x) / per_tile;
-  const int rem = static_cast<int>(blockIdx.x) % per_tile;
+  // Longest-first order: the last query pairs carry the most causal work.
+  const int per_pair = a.Hq * a.B;
+  const int pair = a.npair - 1 - static_cast<int>(blockIdx.x) / per_pair;
+  const int rem = static_cast<int>(blockIdx.x) % per_pair;
   const int b = rem / a.Hq, h = rem % a.Hq, g = h / a.G;
   const bool fa = a.layer_mode == nullptr || a.layer_mode[a.layer] != 0;
-
-  TileIter it_count;
-  it_count.init(a, qt, fa);
-  int n = 0;
-  {
-    int J;
-    uint32_t sm;
-    while (it_count.next(J, sm)) ++n;
-  }
+  const int q0 = pair * 256;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_Q], 1);
@@ -208,21 +159,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[B_KF + s], 1);
       mbar_init(&bars[B_VF + s], 1);
       mbar_init(&bars[B_KE + s], 1);
+      mbar_init(&bars[B_SF + s], 1);
+      mbar_init(&bars[B_PF + s], 128);
     }
-    mbar_init(&bars[B_SF], 1);
-    mbar_init(&bars[B_SFREE], 128);
-    mbar_init(&bars[B_PF], 128);
     mbar_init(&bars[B_OD], 1);
     mbar_init(&bars[B_DRAIN], 1);
     fence_barrier_init();
+  }
+  if (warp == 0) {
+    const int n = fa ? min(2 * pair + 1, a.nkt - 1) + 1 : build_tile_list(a, pair, map, list);
+    if (lane == 0) *nlist = n;
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;         // columns [0, 128)
-  const uint32_t tO = tmem + 128;   // columns [128, 128 + D)
+  const int n = *nlist;
+  auto tile_of = [&](int j, uint32_t& mask) -> int {
+    if (fa) {
+      mask = 0xFFu;
+      return j;
+    }
+    const uint32_t e = list[j];
+    mask = e >> 24;
+    return static_cast<int>(e & 0xFFFFFFu);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -230,18 +192,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars[B_Q], CH * kChunkBytes);
-      for (int c = 0; c < CH; ++c)
-        tma_load_4d(&tm_q, &bars[B_Q], sQ + c * kChunkBytes, c * 64, h, qt * kBM, b);
-      TileIter iter;
-      iter.init(a, qt, fa);
-      int J;
-      uint32_t sm;
+      mbar_arrive_expect_tx(&bars[B_Q], 2 * CH * kChunkBytes);
+      for (int i = 0; i < 2; ++i)
+        for (int c = 0; c < CH; ++c)
+          tma_load_4d(&tm_q, &bars[B_Q], sQ + (i * CH + c) * kChunkBytes, c * 64, h,
+                      q0 + i * kBM, b);
       int issued = 0;
       bool ok = true;
-      for (int it = 0; it < n && iter.next(J, sm); ++it) {
-        const int s = it & 1;
-        if (it >= 2 && !mbar_wait(&bars[B_KE + s], ((it >> 1) - 1) & 1, a.st)) { ok = false; break; }
+      for (int j = 0; j < n; ++j) {
+        const int s = j & 1;
+        uint32_t mask;
+        const int J = tile_of(j, mask);
+        if (j >= 2 && !mbar_wait(&bars[B_KE + s], ((j >> 1) - 1) & 1, a.st)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars[B_KF + s], CH * kChunkBytes);
         for (int c = 0; c < CH; ++c)
           tma_load_4d(&tm_k, &bars[B_KF + s], sK + (s * CH + c) * kChunkBytes, c * 64, g,
@@ -250,15 +212,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < CH; ++c)
           tma_load_4d(&tm_v, &bars[B_VF + s], sV + (s * CH + c) * kChunkBytes, c * 64, g,
                       J * kBN, b);
-        issued = it + 1;
+        issued = j + 1;
       }
       if (!ok) {
         // Let the copies already issued land before the CTA's smem goes away.
         DevStatus drain = a.st;
         drain.spin_ns = 100000000;  // 100 ms
-        for (int it = issued - 2 < 0 ? 0 : issued - 2; it < issued; ++it) {
-          mbar_wait(&bars[B_KF + (it & 1)], (it >> 1) & 1, drain);
-          mbar_wait(&bars[B_VF + (it & 1)], (it >> 1) & 1, drain);
+        mbar_wait(&bars[B_Q], 0, drain);
+        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
+          mbar_wait(&bars[B_KF + (j & 1)], (j >> 1) & 1, drain);
+          mbar_wait(&bars[B_VF + (j & 1)], (j >> 1) & 1, drain);
         }
       }
     }
@@ -268,141 +231,148 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = umma_idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t idesc_o = umma_idesc_bf16(kBM, D, false, true);
       const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      const uint32_t p_addr = smem_u32(sP);
-      bool ok = mbar_wait(&bars[B_Q], 0, a.st);
-      for (int it = 0; ok && it <= n; ++it) {
-        if (it < n) {
-          const int s = it & 1;
-          if (!mbar_wait(&bars[B_KF + s], (it >> 1) & 1, a.st)) { ok = false; break; }
-          if (it >= 1 && !mbar_wait(&bars[B_SFREE], (it - 1) & 1, a.st)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kb = k_addr + s * CH * kChunkBytes;
+      auto issue_s = [&](int i, int s) {
+        const uint32_t qb = q_addr + i * CH * kChunkBytes, kb = k_addr + s * CH * kChunkBytes;
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
-            umma_bf16_ss(tS, umma_smem_desc(q_addr + off, 16, 1024, kSwizzle128B),
-                         umma_smem_desc(kb + off, 16, 1024, kSwizzle128B), idesc_s, ks > 0);
-          }
-          umma_commit(&bars[B_SF]);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
+          umma_bf16_ss(tmem + i * 128, umma_smem_desc(qb + off, 16, 1024, kSwizzle128B),
+                       umma_smem_desc(kb + off, 16, 1024, kSwizzle128B), idesc_s, ks > 0);
         }
-        if (it >= 1) {
-          const int j = it - 1, sj = j & 1;
-          if (!mbar_wait(&bars[B_PF], j & 1, a.st)) { ok = false; break; }
-          if (!mbar_wait(&bars[B_VF + sj], (j >> 1) & 1, a.st)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t vb = v_addr + sj * CH * kChunkBytes;
+      };
+      auto issue_pv = [&](int i, int s, bool acc) {
+        const uint32_t vb = v_addr + s * CH * kChunkBytes;
 #pragma unroll
-          for (int ks = 0; ks < kBN / 16; ++ks) {
-            const uint32_t poff = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
-            umma_bf16_ss(tO, umma_smem_desc(p_addr + poff, 16, 1024, kSwizzle128B),
-                         umma_smem_desc(vb + ks * 16 * 128, kChunkBytes, 1024, kSwizzle128B),
-                         idesc_o, (j > 0 || ks > 0) ? 1u : 0u);
-          }
-          umma_commit(&bars[B_OD]);
-          umma_commit(&bars[B_KE + sj]);
+        for (int ks = 0; ks < kBN / 16; ++ks)
+          umma_bf16_ts(tmem + 256 + i * 128, tmem + i * 128 + ks * 8,
+                       umma_smem_desc(vb + ks * 16 * 128, kChunkBytes, 1024, kSwizzle128B),
+                       idesc_o, (acc || ks > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&bars[B_Q], 0, a.st) && mbar_wait(&bars[B_KF], 0, a.st);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        umma_commit(&bars[B_SF + 0]);
+        issue_s(1, 0);
+        umma_commit(&bars[B_SF + 1]);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int s = j & 1, sn = (j + 1) & 1;
+        const bool more = j + 1 < n;
+        if (!mbar_wait(&bars[B_PF + 0], j & 1, a.st) ||
+            !mbar_wait(&bars[B_VF + s], (j >> 1) & 1, a.st)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(0, s, j > 0);
+        if (more) {
+          if (!mbar_wait(&bars[B_KF + sn], ((j + 1) >> 1) & 1, a.st)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(0, sn);
+          umma_commit(&bars[B_SF + 0]);
+        }
+        if (!mbar_wait(&bars[B_PF + 1], j & 1, a.st)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, s, j > 0);
+        umma_commit(&bars[B_KE + s]);
+        if (more) {
+          issue_s(1, sn);
+          umma_commit(&bars[B_SF + 1]);
         }
       }
+      if (ok) umma_commit(&bars[B_OD]);
       // Every MMA issued by this thread is complete before TMEM is released.
       umma_commit(&bars[B_DRAIN]);
       DevStatus drain = a.st;
       drain.spin_ns = 100000000;
       mbar_wait(&bars[B_DRAIN], 0, drain);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
+    const int i = (warp - 4) >> 2;           // query tile 0 or 1
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;       // row within the tile
-    const int t_row = qt * kBM + r;
+    const int t_row = q0 + i * kBM + r;
+    const int qs = (i * kBM + r) >> 6;       // 64-row sub-block within the pair
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t p_addr = smem_u32(sP);
+    const uint32_t tS = tmem + lane_off + i * 128;
+    const uint32_t tO = tmem + lane_off + 256 + i * 128;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    TileIter iter;
-    iter.init(a, qt, fa);
-    int J;
-    uint32_t sm;
-    for (int it = 0; it < n && iter.next(J, sm); ++it) {
-      if (!mbar_wait(&bars[B_SF], it & 1, a.st)) { ok = false; break; }
+    for (int j = 0; j < n; ++j) {
+      uint32_t mask;
+      const int J = tile_of(j, mask);
+      if (!mbar_wait(&bars[B_SF + i], j & 1, a.st)) { ok = false; break; }
       tc_fence_after();
       float x[kBN];
+      {
+        uint32_t v[kBN / 32][32];
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + lane_off + c * 32, v);
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, v[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]) * a.scale_log2;
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[B_SFREE]);
-
-      const bool diag = (J == qt);
-      if (diag || sm != 0xFu) {
-        const int qhalf = r >> 6;
+        for (int c = 0; c < kBN / 32; ++c)
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          const bool causal_ok = !diag || (J * kBN + c <= t_row);
-          const bool blk_ok = (sm >> (qhalf * 2 + (c >> 6))) & 1u;
-          if (!(causal_ok && blk_ok)) x[c] = -INFINITY;
-        }
+          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[c][e]);
+      }
+      const uint32_t sub = (mask >> (qs * 2)) & 3u;
+      if (J * kBN + kBN - 1 > t_row || sub != 3u) {
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          if (J * kBN + c > t_row || !((sub >> (c >> 6)) & 1u)) x[c] = -INFINITY;
       }
       float mt = x[0];
 #pragma unroll
       for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, x[c]);
-      const float m_new = fmaxf(m_run, mt);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2(m_run - m_use);
+      const float m_tile = mt * a.scale_log2;
+      const bool grow = m_tile > m_run + kRescaleLog2;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = ex2(m_run - m_tile);
+        l_run *= alpha;
+        m_run = m_tile;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       float rs = 0.f;
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) {
-        x[c] = ex2(x[c] - m_use);
-        rs += x[c];
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(fmaf(x[c * 32 + 2 * e], a.scale_log2, -m_use));
+          const float p1 = ex2(fmaf(x[c * 32 + 2 * e + 1], a.scale_log2, -m_use));
+          rs += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + c * 16, pk);   // P_i over S_i's first 64 columns
       }
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-
-      if (it >= 1 && !mbar_wait(&bars[B_OD], (it - 1) & 1, a.st)) { ok = false; break; }
-      // P row -> shared memory, bf16, 128-byte swizzle (16-byte unit u ^ (row & 7)).
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O_i is stable: S_i(j) completing implies PV_i(j-1) completed, and
+        // PV_i(j) waits for this warpgroup's arrival below.
 #pragma unroll
-      for (int u = 0; u < kBN / 8; ++u) {
-        const uint32_t w0 = pack_bf16x2(x[u * 8 + 0], x[u * 8 + 1]);
-        const uint32_t w1 = pack_bf16x2(x[u * 8 + 2], x[u * 8 + 3]);
-        const uint32_t w2 = pack_bf16x2(x[u * 8 + 4], x[u * 8 + 5]);
-        const uint32_t w3 = pack_bf16x2(x[u * 8 + 6], x[u * 8 + 7]);
-        const uint32_t addr = p_addr + (u >> 3) * kChunkBytes + r * 128 +
-                              ((((u & 7) ^ (r & 7))) << 4);
-        st_shared_v4(addr, w0, w1, w2, w3);
-      }
-      fence_proxy_async_smem();
-      if (it >= 1) {
-        tc_fence_after();
-        if (!__all_sync(0xffffffffu, alpha == 1.f)) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tO + c * 32, v);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tO + lane_off + c * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            tmem_st32(tO + lane_off + c * 32, v);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+          tmem_st32(tO + c * 32, v);
         }
       }
+      l_run += rs;
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[B_PF]);
+      mbar_arrive(&bars[B_PF + i]);
     }
 
     // ------------------------------------------------------------ epilogue
     const size_t row_elem = ((static_cast<size_t>(b) * a.T + t_row) * a.Hq + h) * D;
     const bool valid = t_row < a.T;
-    if (n > 0 && ok && mbar_wait(&bars[B_OD], (n - 1) & 1, a.st)) {
+    if (n > 0 && ok && mbar_wait(&bars[B_OD], 0, a.st)) {
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tO + lane_off + c * 32, v);
+        tmem_ld32(tO + c * 32, v);
         tmem_wait_ld();
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(a.o + row_elem + c * 32);
@@ -447,7 +417,8 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
   a.G = p.Hq / p.Hkv;
-  a.nqt = (p.T + kBM - 1) / kBM;
+  a.npair = (p.T + 255) / 256;
+  a.nkt = (p.T + kBN - 1) / kBN;
   a.block = p.block;
   a.nqb = p.nqb;
   a.nkb = (p.T + p.block - 1) / p.block;
@@ -459,7 +430,7 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   a.o = p.o;
   a.lse = p.lse;
   a.st = p.st;
-  const dim3 grid(static_cast<unsigned>(a.nqt) * p.Hq * p.B);
+  const dim3 grid(static_cast<unsigned>(a.npair) * p.Hq * p.B);
   if (p.d == 64) {
     const int smem = Smem<64>::ALLOC;
     cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
