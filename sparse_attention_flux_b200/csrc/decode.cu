@@ -7,18 +7,21 @@
 // Decode is bound by HBM bandwidth (section 1 of the same summary), so the
 // kernel is built around the KV stream:
 //   * grid (split, kv head, sequence); each CTA streams one chunk of one
-//     (sequence, kv head) and serves all G = Hq/Hkv query heads of that group
-//     from the single read;
-//   * 64-token K and V tiles arrive by TMA (128-byte swizzle, so that the
-//     per-token and per-channel shared-memory reads are conflict-free) into a
-//     4-stage ring guarded by mbarriers;
-//   * scores: 4 threads per token, fp32 FMAs on bf16 data widened in
-//     registers, a 2-step shuffle to combine the quarters, online softmax in
-//     the log2 domain;
-//   * values: each thread owns 8 channels of all G heads for a subset of the
-//     tile's tokens; the subsets are combined once per CTA;
-//   * the last CTA of each (sequence, kv head) -- found by an atomic ticket,
-//     no spin -- merges the partial (o, m, l) of every active split.
+//     (sequence, kv head) and serves all G = Hq/Hkv query heads of the group
+//     from that single read;
+//   * a producer warp moves 64-token K and V tiles by TMA (128-byte swizzle)
+//     into a 3-stage ring; four compute warps each own a 16-token slice of
+//     every tile, so the loop has no block barrier: a stage is released by an
+//     mbarrier that counts the four warps;
+//   * per warp, the group's scores S[G x 16] = Q K^T and values O += P V are
+//     16x8x16 warp MMAs (bf16 in, fp32 accumulate) fed by ldmatrix straight
+//     from the swizzled tiles -- the G query heads fill rows 0..G-1 of the
+//     16-row operand; online softmax in the log2 domain on the accumulator
+//     fragments, O rescaled only when a row max grows by more than 2^8;
+//   * the four warps' partials are merged in shared memory, then the last CTA
+//     of each (sequence, kv head) -- found by an atomic ticket, no spin --
+//     merges the partial (o, m, l) of every active split.
+// About 110 registers and 97 KB of shared memory: two CTAs per SM.
 #include <algorithm>
 
 #include "common.cuh"
@@ -28,9 +31,11 @@ namespace flux {
 
 namespace {
 
-constexpr int kTok = 64;        // tokens per tile
-constexpr int kStages = 4;
-constexpr int kThreads = 256;
+constexpr int kTok = 64;        // tokens per tile (4 warps x 16)
+constexpr int kStages = 3;
+constexpr int kComputeWarps = 4;
+constexpr int kThreads = 32 * (kComputeWarps + 1);
+constexpr float kRescaleLog2 = 8.f;
 
 template <int D>
 struct DSmem {
@@ -38,12 +43,13 @@ struct DSmem {
   static constexpr int BOX = kTok * 128;           // one box: 64 tokens x 128 bytes
   static constexpr int KT = CH * BOX;              // K tile bytes
   static constexpr int STAGE = 2 * KT;             // K + V
-  static constexpr int P = kStages * STAGE;        // p[64][4] fp32
-  static constexpr int RED = P + kTok * 16;        // [8 warps][4] fp32
-  static constexpr int BARS = RED + 8 * 4 * 4;
-  static constexpr int FLAG = BARS + kStages * 8;
+  static constexpr int BARS = kStages * STAGE;     // full[kStages], empty[kStages]
+  static constexpr int FLAG = BARS + 2 * kStages * 8;
   static constexpr int TOTAL = FLAG + 16;
   static constexpr int ALLOC = TOTAL + 1024;
+  // After the stream: per-warp partials [warp][4 heads] m, l and o[warp][4][D].
+  static constexpr int CM = 0, CL = CM + kComputeWarps * 4 * 4, CO = CL + kComputeWarps * 4 * 4;
+  static_assert(CO + kComputeWarps * 4 * D * 4 <= BARS, "combine area must fit in the ring");
 };
 
 struct Range {
@@ -80,20 +86,17 @@ __device__ __forceinline__ Range split_range(const DecodeLaunch& a, bool fa, int
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecodeLaunch a) {
   using L = DSmem<D>;
-  constexpr int QW = D / 4;          // channels per quarter-thread in the score phase
-  constexpr int NCH = D / 8;         // 8-channel units per row
-  constexpr int NSUB = kThreads / NCH;   // token subsets in the value phase
-  constexpr int TPS = kTok / NSUB;       // tokens per thread per tile in the value phase
+  constexpr int KS = D / 16;        // k-steps of the score MMA
+  constexpr int NT = D / 8;         // n-tiles of the value MMA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  float* p_s = reinterpret_cast<float*>(smem + L::P);
-  float* red = reinterpret_cast<float*>(smem + L::RED);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
+  uint64_t* empty = full + kStages;
   int* flag = reinterpret_cast<int*>(smem + L::FLAG);
 
   const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -108,193 +111,186 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntiles = (rg.end - rg.start + kTok - 1) / kTok;
 
   if (tid == 0) {
-    for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kComputeWarps);
+    }
     fence_barrier_init();
   }
   __syncthreads();
 
-  auto issue = [&](int k) {
-    const int st = k % kStages;
-    uint8_t* kb = smem + st * L::STAGE;
-    uint8_t* vb = kb + L::KT;
-    mbar_arrive_expect_tx(&full[st], 2 * L::KT);
-    const int tok = rg.start + k * kTok;
-    for (int c = 0; c < L::CH; ++c) {
-      tma_load_4d(&tm_k, &full[st], kb + c * L::BOX, c * 64, g, tok, b);
-      tma_load_4d(&tm_v, &full[st], vb + c * L::BOX, c * 64, g, tok, b);
-    }
-  };
-  if (tid == 0 && ntiles > 0) {
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    for (int k = 0; k < kStages && k < ntiles; ++k) issue(k);
-  }
-
-  // Query registers for the score phase: G heads x QW channels, pre-scaled
-  // into the log2 domain.
-  const int tj = tid >> 2, qd = tid & 3;
-  float qr[G][QW];
-  {
-    const float sl2 = a.scale * 1.4426950408889634f;
+  const int gq = lane >> 2, tq = lane & 3;   // fragment row (head) and column pair
+  float m_run = -INFINITY, l_part = 0.f;
+  float oacc[NT][4];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      const uint4* src = reinterpret_cast<const uint4*>(
-          a.q + (static_cast<size_t>(b) * a.Hq + g * G + hh) * D + qd * QW);
-#pragma unroll
-      for (int u = 0; u < QW / 8; ++u) {
-        const uint4 w = src[u];
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          qr[hh][u * 8 + 2 * e] = bf16lo_to_f32(ws[e]) * sl2;
-          qr[hh][u * 8 + 2 * e + 1] = bf16hi_to_f32(ws[e]) * sl2;
-        }
-      }
-    }
-  }
-
-  float m_run[G], acc[G][8];
-  float l_part = 0.f;
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    m_run[hh] = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
-  }
-  const int vch = tid % NCH, vsub = tid / NCH;
+  for (int n = 0; n < NT; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
   bool ok = true;
-  int consumed = 0;
 
-  for (int k = 0; k < ntiles; ++k) {
-    const int st = k % kStages;
-    if (!mbar_wait(&full[st], (k / kStages) & 1, a.st)) { ok = false; break; }
-    const uint32_t kb = smem_u32(smem + st * L::STAGE);
-    const uint32_t vb = kb + L::KT;
-    const int tok0 = rg.start + k * kTok;
-
-    // ---- scores: token tj, channel quarter qd
-    float dot[G];
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) dot[hh] = 0.f;
-#pragma unroll
-    for (int u = 0; u < QW / 8; ++u) {
-      const int unit = qd * (QW / 8) + u;         // 16-byte unit along the row (0 .. D/8-1)
-      const int box = unit >> 3, uu = unit & 7;
-      const uint4 w = ld_shared_v4(kb + box * L::BOX + tj * 128 + ((uu ^ (tj & 7)) << 4));
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float k0 = bf16lo_to_f32(ws[e]), k1 = bf16hi_to_f32(ws[e]);
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          dot[hh] = fmaf(qr[hh][u * 8 + 2 * e], k0, dot[hh]);
-          dot[hh] = fmaf(qr[hh][u * 8 + 2 * e + 1], k1, dot[hh]);
+  if (warp == kComputeWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && ntiles > 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int issued = 0;
+      for (int k = 0; k < ntiles; ++k) {
+        const int st = k % kStages;
+        if (k >= kStages && !mbar_wait(&empty[st], ((k / kStages) - 1) & 1, a.st)) {
+          ok = false;
+          break;
         }
+        uint8_t* kb = smem + st * L::STAGE;
+        uint8_t* vb = kb + L::KT;
+        mbar_arrive_expect_tx(&full[st], 2 * L::KT);
+        const int tok = rg.start + k * kTok;
+        for (int c = 0; c < L::CH; ++c) {
+          tma_load_4d(&tm_k, &full[st], kb + c * L::BOX, c * 64, g, tok, b);
+          tma_load_4d(&tm_v, &full[st], vb + c * L::BOX, c * 64, g, tok, b);
+        }
+        issued = k + 1;
+      }
+      if (!ok) {
+        // Let the copies still in flight land before the CTA's smem goes away.
+        DevStatus drain = a.st;
+        drain.spin_ns = 100000000;
+        for (int k = max(0, issued - kStages); k < issued; ++k)
+          mbar_wait(&full[k % kStages], (k / kStages) & 1, drain);
       }
     }
+  } else if (ntiles > 0) {
+    // ------------------------------------------------------------ compute warps
+    // Q fragments (rows = the group's G heads, zero beyond), A of the score MMA.
+    uint32_t qa[KS][4];
+    {
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          a.q + (static_cast<size_t>(b) * a.Hq + g * G + (gq < G ? gq : 0)) * D);
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      dot[hh] += __shfl_xor_sync(0xffffffffu, dot[hh], 1);
-      dot[hh] += __shfl_xor_sync(0xffffffffu, dot[hh], 2);
-    }
-    const bool valid = (tok0 + tj < rg.end) && (qd < G);
-    float sc = -INFINITY;
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-      if (hh == qd && valid) sc = dot[hh];
-    float mx = sc;
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    if (lane < 4) red[warp * 4 + lane] = mx;
-    __syncthreads();
-    float alpha[G], m_use[G];
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      float t = red[hh];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) t = fmaxf(t, red[w * 4 + hh]);
-      const float m_new = fmaxf(m_run[hh], t);
-      m_use[hh] = (m_new == -INFINITY) ? 0.f : m_new;
-      alpha[hh] = ex2(m_run[hh] - m_use[hh]);
-      m_run[hh] = m_new;
-    }
-    float my_m = 0.f, my_alpha = 1.f;
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-      if (hh == qd) { my_m = m_use[hh]; my_alpha = alpha[hh]; }
-    const float p = valid ? ex2(sc - my_m) : 0.f;
-    l_part = l_part * my_alpha + p;
-    p_s[tj * 4 + qd] = p;
-    __syncthreads();
-
-    // ---- values: channels 8*vch .. +7, tokens vsub + NSUB*n
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[hh][e] *= alpha[hh];
-#pragma unroll
-    for (int n = 0; n < TPS; ++n) {
-      const int j = vsub + NSUB * n;
-      const int box = vch >> 3, uu = vch & 7;
-      const uint4 w = ld_shared_v4(vb + box * L::BOX + j * 128 + ((uu ^ (j & 7)) << 4));
-      const float4 pj = *reinterpret_cast<const float4*>(p_s + j * 4);
-      const float pv[4] = {pj.x, pj.y, pj.z, pj.w};
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float v0 = bf16lo_to_f32(ws[e]), v1 = bf16hi_to_f32(ws[e]);
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          acc[hh][2 * e] = fmaf(pv[hh], v0, acc[hh][2 * e]);
-          acc[hh][2 * e + 1] = fmaf(pv[hh], v1, acc[hh][2 * e + 1]);
-        }
+      for (int ks = 0; ks < KS; ++ks) {
+        qa[ks][0] = gq < G ? qrow[ks * 8 + tq] : 0u;
+        qa[ks][2] = gq < G ? qrow[ks * 8 + 4 + tq] : 0u;
+        qa[ks][1] = qa[ks][3] = 0u;
       }
     }
-    __syncthreads();  // stage st and p_s are free again
-    consumed = k + 1;
-    if (tid == 0 && k + kStages < ntiles) issue(k + kStages);
-  }
-  if (!ok && tid == 0) {
-    // Let the copies still in flight land before the CTA's smem goes away.
-    DevStatus drain = a.st;
-    drain.spin_ns = 100000000;
-    const int last = min(ntiles, consumed + kStages);
-    for (int k = consumed; k < last; ++k) mbar_wait(&full[k % kStages], (k / kStages) & 1, drain);
+    const float sl2 = a.scale * 1.4426950408889634f;
+    const int mrow = lane & 7, msel = lane >> 3;     // ldmatrix row and matrix index
+    const int wtok = warp * 16;
+    for (int k = 0; k < ntiles; ++k) {
+      const int st = k % kStages;
+      if (!mbar_wait(&full[st], (k / kStages) & 1, a.st)) { ok = false; break; }
+      const uint32_t kb = smem_u32(smem + st * L::STAGE);
+      const uint32_t vb = kb + L::KT;
+      // ---- scores: S[head][token] for this warp's 16 tokens (two n-tiles of 8)
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int tok = wtok + (msel >> 1) * 8 + mrow;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int uu = 2 * ks + (msel & 1);
+          const uint32_t addr = kb + (uu >> 3) * L::BOX + tok * 128 + (((uu & 7) ^ (tok & 7)) << 4);
+          uint32_t b00, b01, b10, b11;
+          ldmatrix_x4(addr, b00, b01, b10, b11);
+          mma_bf16_16816(sc[0], qa[ks], b00, b01);
+          mma_bf16_16816(sc[1], qa[ks], b10, b11);
+        }
+      }
+      // ---- online softmax on the fragment: row gq, tokens 8n + 2tq + e
+      const int tok0 = rg.start + k * kTok + wtok + 2 * tq;
+      float x[4];
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          x[n * 2 + e] = (gq < G && tok0 + 8 * n + e < rg.end) ? sc[n][e] : -INFINITY;
+      float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+      const float m_tile = mt * sl2;
+      const bool grow = m_tile > m_run + kRescaleLog2;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = ex2(m_run - m_tile);
+        l_part *= alpha;
+        m_run = m_tile;
+      }
+      if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          oacc[n][0] *= alpha;
+          oacc[n][1] *= alpha;
+        }
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        p[e] = ex2(fmaf(x[e], sl2, -m_use));
+        l_part += p[e];
+      }
+      const uint32_t pa[4] = {pack_bf16x2(p[0], p[1]), 0u, pack_bf16x2(p[2], p[3]), 0u};
+      // ---- values: O[head][d] += P[head][16 tokens] V[16 tokens][d]
+      {
+        const int tok = wtok + (msel & 1) * 8 + mrow;
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          const int uu = 2 * np + (msel >> 1);
+          const uint32_t addr = vb + (uu >> 3) * L::BOX + tok * 128 + (((uu & 7) ^ (tok & 7)) << 4);
+          uint32_t b0a, b1a, b0b, b1b;
+          ldmatrix_x4_trans(addr, b0a, b1a, b0b, b1b);
+          mma_bf16_16816(oacc[2 * np], pa, b0a, b1a);
+          mma_bf16_16816(oacc[2 * np + 1], pa, b0b, b1b);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
   }
   __syncthreads();
 
-  // ---- combine within the CTA: l per head, acc over the NSUB token subsets
-  float* comb = reinterpret_cast<float*>(smem);  // [NSUB][G][D], reuses the stage ring
-  {
-    float lp = l_part;
-    lp += __shfl_xor_sync(0xffffffffu, lp, 4);
-    lp += __shfl_xor_sync(0xffffffffu, lp, 8);
-    lp += __shfl_xor_sync(0xffffffffu, lp, 16);
-    if (lane < 4) red[warp * 4 + lane] = lp;
+  // ---- merge the four warps' partials in shared memory (the ring is free now)
+  float* cm = reinterpret_cast<float*>(smem + L::CM);
+  float* cl = reinterpret_cast<float*>(smem + L::CL);
+  float* co = reinterpret_cast<float*>(smem + L::CO);
+  if (warp < kComputeWarps) {
+    float lq = l_part;
+    lq += __shfl_xor_sync(0xffffffffu, lq, 1);
+    lq += __shfl_xor_sync(0xffffffffu, lq, 2);
+    if (gq < 4) {
+      if (tq == 0) {
+        cm[warp * 4 + gq] = (ntiles > 0) ? m_run : -INFINITY;
+        cl[warp * 4 + gq] = (ntiles > 0) ? lq : 0.f;
+      }
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) comb[(vsub * G + hh) * D + vch * 8 + e] = acc[hh][e];
+      for (int n = 0; n < NT; ++n) {
+        co[(warp * 4 + gq) * D + 8 * n + 2 * tq] = oacc[n][0];
+        co[(warp * 4 + gq) * D + 8 * n + 2 * tq + 1] = oacc[n][1];
+      }
+    }
   }
   __syncthreads();
   const size_t grp = static_cast<size_t>(b) * a.Hq + g * G;  // first query head of the group
   if (rg.end > rg.start) {
     for (int idx = tid; idx < G * D; idx += kThreads) {
       const int hh = idx / D, c = idx % D;
-      float t = 0.f;
-      for (int sidx = 0; sidx < NSUB; ++sidx) t += comb[(sidx * G + hh) * D + c];
-      a.part_o[((grp + hh) * a.nsplit + i) * D + c] = t;
-    }
-    if (tid < G) {
-      float l = 0.f;
-      for (int w = 0; w < 8; ++w) l += red[w * 4 + tid];
-      a.part_ml[((grp + tid) * a.nsplit + i) * 2 + 0] = m_run[tid];
-      a.part_ml[((grp + tid) * a.nsplit + i) * 2 + 1] = l;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, cm[w * 4 + hh]);
+      float O = 0.f, Lsum = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kComputeWarps; ++w) {
+          const float wt = ex2(cm[w * 4 + hh] - M);
+          O += wt * co[(w * 4 + hh) * D + c];
+          Lsum += wt * cl[w * 4 + hh];
+        }
+      }
+      a.part_o[((grp + hh) * a.nsplit + i) * D + c] = O;
+      if (c == 0) {
+        a.part_ml[((grp + hh) * a.nsplit + i) * 2 + 0] = M;
+        a.part_ml[((grp + hh) * a.nsplit + i) * 2 + 1] = Lsum;
+      }
     }
   }
 
-  // ---- ticket: the last CTA of this (sequence, kv head) merges
+  // ---- ticket: the last CTA of this (sequence, kv head) merges the splits
   __threadfence();
   __syncthreads();
   if (tid == 0) {
