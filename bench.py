@@ -278,22 +278,22 @@ def run_flux(args, rank, world, dev_index):
     for _ in range(args.warmup):
         wl.step()
     ctx.check()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(2)]
-    fa_ms, sa_ms = [], []
+    # Per-kernel CUDA events on the launching (current) stream, read after the
+    # loop so that no host synchronisation sits inside the timed region.
+    new_ev = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [[[new_ev(), new_ev()] for _ in range(2)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev_index) as clk:
-        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start, stop = new_ev(), new_ev()
         start.record()
-        for _ in range(args.steps):
-            wl.step(ev)
-            # per-kernel durations from events on the launching (current) stream
-            stop.record()
-            stop.synchronize()
-            fa_ms.append(ev[0][0].elapsed_time(ev[0][1]))
-            sa_ms.append(ev[1][0].elapsed_time(ev[1][1]))
+        for k in range(args.steps):
+            wl.step(evs[k])
+        stop.record()
         torch.cuda.synchronize()
     barrier()
+    fa_ms = [e[0][0].elapsed_time(e[0][1]) for e in evs]
+    sa_ms = [e[1][0].elapsed_time(e[1][1]) for e in evs]
     total_ms = start.elapsed_time(stop)
     ctx.check()
     clocks = clk.summary()
@@ -332,18 +332,16 @@ def run_flux(args, rank, world, dev_index):
         for s in range(min(3, dw.steps)):
             dw.step(s)
         ctx.check()
-        fev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-        fa_dec_ms = []
+        fevs = [(new_ev(), new_ev()) for _ in range(dw.steps)]
         barrier()
         torch.cuda.synchronize()
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0, d1 = new_ev(), new_ev()
         d0.record()
         for s in range(dw.steps):
-            dw.step(s, fev)
-            fev[1].synchronize()
-            fa_dec_ms.append(fev[0].elapsed_time(fev[1]))
+            dw.step(s, fevs[s])
         d1.record()
         d1.synchronize()
+        fa_dec_ms = [a_.elapsed_time(b_) for a_, b_ in fevs]
         ctx.check()
         dec_ms = max_over_ranks(d0.elapsed_time(d1) / dw.steps)
         dec_gbs = dw.bytes_per_step * world / (dec_ms * 1e-3) / 1e9

@@ -18,9 +18,10 @@
 //     from the swizzled tiles -- the G query heads fill rows 0..G-1 of the
 //     16-row operand; online softmax in the log2 domain on the accumulator
 //     fragments, O rescaled only when a row max grows by more than 2^8;
-//   * the four warps' partials are merged in shared memory, then the last CTA
-//     of each (sequence, kv head) -- found by an atomic ticket, no spin --
-//     merges the partial (o, m, l) of every active split.
+//   * the four warps' partials are merged in shared memory, then the last
+//     active CTA of each (sequence, kv head) -- found by an atomic ticket, no
+//     spin -- merges the partial (o, m, l) of every active split; splits past
+//     the active range (most of an SA layer's grid) exit at entry.
 // About 110 registers and 97 KB of shared memory: two CTAs per SM.
 #include <algorithm>
 
@@ -109,6 +110,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   const Range rg = split_range(a, fa, s, i);
   const int ntiles = (rg.end - rg.start + kTok - 1) / kTok;
+  const size_t grp = static_cast<size_t>(b) * a.Hq + g * G;  // first query head of the group
+  if (ntiles == 0) {
+    // Splits past the active range exit at once (SA layers use only a few);
+    // with no visible token at all, split 0 writes the zero output.
+    if (i == 0 && rg.n_active == 0) {
+      for (int idx = tid; idx < G * D; idx += kThreads) {
+        reinterpret_cast<__nv_bfloat16*>(a.o)[grp * D + idx] = __float2bfloat16_rn(0.f);
+        if (idx % D == 0 && a.lse) a.lse[grp + idx / D] = -INFINITY;
+      }
+    }
+    return;
+  }
 
   if (tid == 0) {
     for (int st = 0; st < kStages; ++st) {
@@ -266,8 +279,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   __syncthreads();
-  const size_t grp = static_cast<size_t>(b) * a.Hq + g * G;  // first query head of the group
-  if (rg.end > rg.start) {
+  {
     for (int idx = tid; idx < G * D; idx += kThreads) {
       const int hh = idx / D, c = idx % D;
       float M = -INFINITY;
@@ -295,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   if (tid == 0) {
     const int old = atomicAdd(&a.tickets[b * a.Hkv + g], 1);
-    *flag = (old == static_cast<int>(gridDim.x) - 1);
+    *flag = (old == rg.n_active - 1);
   }
   __syncthreads();
   if (!*flag) return;

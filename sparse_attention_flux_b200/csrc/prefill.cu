@@ -319,9 +319,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kBN; ++c)
           if (J * kBN + c > t_row || !((sub >> (c >> 6)) & 1u)) x[c] = -INFINITY;
       }
-      float mt = x[0];
+      // Row max with 8 independent accumulators (a 127-deep chain otherwise).
+      float mx[8];
 #pragma unroll
-      for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, x[c]);
+      for (int e = 0; e < 8; ++e) mx[e] = x[e];
+#pragma unroll
+      for (int c = 8; c < kBN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_tile = mt * a.scale_log2;
       const bool grow = m_tile > m_run + kRescaleLog2;
       float alpha = 1.f;
@@ -331,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_tile;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float rs = 0.f;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial row sums
 #pragma unroll
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t pk[16];
@@ -339,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e) {
           const float p0 = ex2(fmaf(x[c * 32 + 2 * e], a.scale_log2, -m_use));
           const float p1 = ex2(fmaf(x[c * 32 + 2 * e + 1], a.scale_log2, -m_use));
-          rs += p0 + p1;
+          rs[e & 3] += p0 + p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);   // P_i over S_i's first 64 columns
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st32(tO + c * 32, v);
         }
       }
-      l_run += rs;
+      l_run += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[B_PF + i]);
