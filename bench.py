@@ -145,6 +145,31 @@ class ClockSampler:
         return out
 
 
+# --------------------------------------------------------------------------- ranks
+
+def dist_barrier(world: int) -> None:
+    """Barrier across ranks (no-op for one process)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of a per-rank time over all ranks (the timing the contract asks for)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float, scale: float = 1e12) -> float:
+    """Aggregate throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms * 1e-3) / scale
+
+
 # --------------------------------------------------------------------------- flux arm
 
 class PrefillWorkload:
@@ -264,16 +289,8 @@ def run_flux(args, rank, world, dev_index):
     from sparse_attention_flux_b200 import synth
     wl = PrefillWorkload(ctx, synth.seed_for(1) + 1000 * rank, dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = lambda: dist_barrier(world)
+    ranks_max = lambda x: max_over_ranks(x, world, dev)
 
     for _ in range(args.warmup):
         wl.step()
@@ -297,9 +314,9 @@ def run_flux(args, rank, world, dev_index):
     total_ms = start.elapsed_time(stop)
     ctx.check()
     clocks = clk.summary()
-    total_ms = max_over_ranks(total_ms)
+    total_ms = ranks_max(total_ms)
     ms_per_step = total_ms / args.steps
-    value = wl.flops * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_rate(wl.flops, world, ms_per_step)
 
     # e2e: host buffers in and out through the same public API
     for _ in range(max(1, args.warmup // 2)):
@@ -313,8 +330,8 @@ def run_flux(args, rank, world, dev_index):
         wl.step_e2e()
     s1.record()
     s1.synchronize()
-    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / e2e_steps)
-    e2e_value = wl.flops * world / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = ranks_max(s0.elapsed_time(s1) / e2e_steps)
+    e2e_value = whole_job_rate(wl.flops, world, e2e_ms)
 
     h2d_bytes, d2h_bytes, launches = wl.h2d_bytes, wl.d2h_bytes, wl.launches * args.steps
     fa_avg = statistics.mean(fa_ms)
@@ -343,8 +360,8 @@ def run_flux(args, rank, world, dev_index):
         d1.synchronize()
         fa_dec_ms = [a_.elapsed_time(b_) for a_, b_ in fevs]
         ctx.check()
-        dec_ms = max_over_ranks(d0.elapsed_time(d1) / dw.steps)
-        dec_gbs = dw.bytes_per_step * world / (dec_ms * 1e-3) / 1e9
+        dec_ms = ranks_max(d0.elapsed_time(d1) / dw.steps)
+        dec_gbs = whole_job_rate(dw.bytes_per_step, world, dec_ms, 1e9)
         fa_dec_avg = statistics.mean(fa_dec_ms)
         fa_dec_gbs = dw.bytes_fa / (fa_dec_avg * 1e-3) / 1e9
         dec = {
