@@ -37,10 +37,12 @@ def rng(seed: int) -> np.random.Generator:
 
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 values to bf16 (nearest even) and return the 16-bit patterns."""
-    u = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return rounded.astype(np.uint16)
+    """Round finite fp32 values to bf16 (nearest even) and return the 16-bit patterns.
+
+    uint32 arithmetic is exact here: a finite value's pattern plus 0x8000 stays
+    below 2^32."""
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32)
+    return ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
