@@ -14,6 +14,8 @@
  *   flux_build_block_index     block mask                   -> CSR row_ptr/col
  *   flux_attn_prefill          one layer, FA or SA per layer_mode[layer]
  *   flux_attn_decode           one layer, one new token per sequence
+ *   flux_kv_write              append / fill a full cache or an SA layer's ring
+ *   flux_attn_decode_sa_compact  SA decode over the ring (sink + last W blocks)
  *
  * Conventions shared by every entry point
  *   - Every tensor pointer is a DEVICE pointer owned by the caller; the
@@ -174,6 +176,41 @@ int flux_attn_decode(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_cache,
                      const uint8_t* layer_mode, int layer,
                      int sink_blocks, int window_blocks, int block, float scale,
                      flux_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * KV-cache writes, and decode over the compact SA cache (gist.science summary
+ * section 2, "efficient deployment": SA layers keep only the minimal KV cache
+ * -- the sink blocks and the last W blocks -- and never read the history).
+ *
+ * flux_kv_write copies the tokens at positions [s - n_src, s) of each sequence
+ * (s = seqlens[b], the length AFTER the write) from k_src/v_src
+ * [B, n_src, Hkv, d] bf16 into a cache:
+ *   window_blocks == 0: a full cache [B, cache_rows, Hkv, d]; row = position
+ *     (an FA layer's per-step append, n_src = 1);
+ *   window_blocks  > 0: the compact ring of an SA layer, [B, cache_rows, Hkv, d]
+ *     with cache_rows = (sink_blocks + window_blocks) * block: rows
+ *     [0, sink*block) hold the sink tokens, block j >= sink_blocks lives in
+ *     slot j mod window_blocks at rows (sink_blocks + j mod W) * block + ...
+ *     Only tokens still live at length s are written (so a whole prompt,
+ *     n_src = T, fills the ring with its sink and last W blocks).
+ * Hkv * d must be a multiple of 8.  A seqlens entry below n_src (or above
+ * cache_rows for a full cache) skips that sequence and sets the error word.
+ *
+ * flux_attn_decode_sa_compact is flux_attn_decode for an SA layer whose cache
+ * is that ring: the same tokens (blocks j < sink or j >= ceil(s/block) - W),
+ * hence the same result as SA decode over the full cache, read from
+ * (sink + W) * block rows per sequence.  block must be a multiple of 64;
+ * seqlens[b] may exceed the ring size (it is the sequence length). */
+int flux_kv_write(flux_ctx* ctx, const uint16_t* k_src, const uint16_t* v_src, int n_src,
+                  const int32_t* seqlens, int B, int Hkv, int d,
+                  uint16_t* k_cache, uint16_t* v_cache, int cache_rows,
+                  int sink_blocks, int window_blocks, int block, flux_stream_t stream);
+
+int flux_attn_decode_sa_compact(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_ring,
+                                const uint16_t* v_ring, const int32_t* seqlens,
+                                uint16_t* o, float* lse, int B, int Hq, int Hkv, int d,
+                                int sink_blocks, int window_blocks, int block, float scale,
+                                flux_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * Decode attention that allocates nothing.  The pages have no counterpart of

@@ -358,9 +358,87 @@ int flux_attn_decode(flux_ctx* c, const uint16_t* q, const uint16_t* k_cache,
   p.part_o = static_cast<float*>(c->workspace);
   p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
   p.tickets = c->tickets;
+  p.compact = 0;
   p.st = status_of(c);
   const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode: launch");
+}
+
+int flux_kv_write(flux_ctx* c, const uint16_t* k_src, const uint16_t* v_src, int n_src,
+                  const int32_t* seqlens, int B, int Hkv, int d, uint16_t* k_cache,
+                  uint16_t* v_cache, int cache_rows, int sink_blocks, int window_blocks,
+                  int block, flux_stream_t stream) {
+  if (!c || !k_src || !v_src || !seqlens || !k_cache || !v_cache)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_kv_write: null pointer argument");
+  if (n_src < 1 || B < 1 || Hkv < 1 || d < 1 || cache_rows < 1 || sink_blocks < 0 ||
+      window_blocks < 0 || block < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_kv_write: bad sizes");
+  if ((static_cast<long long>(Hkv) * d) % 8 != 0)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_kv_write: Hkv * d must be a multiple of 8");
+  if (window_blocks > 0 && static_cast<long long>(sink_blocks + window_blocks) * block != cache_rows)
+    return fail(FLUX_ERR_SHAPE, "flux_kv_write: ring cache_rows must be (sink + window) * block");
+  if (!aligned16(k_src) || !aligned16(v_src) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_kv_write: tensors must be 16-byte aligned");
+  const cudaError_t e = flux::launch_ring_write(
+      k_src, v_src, n_src, seqlens, B, Hkv, d, k_cache, v_cache, sink_blocks, window_blocks,
+      window_blocks > 0 ? block : cache_rows, c->err, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_kv_write: launch");
+}
+
+int flux_attn_decode_sa_compact(flux_ctx* c, const uint16_t* q, const uint16_t* k_ring,
+                                const uint16_t* v_ring, const int32_t* seqlens, uint16_t* o,
+                                float* lse, int B, int Hq, int Hkv, int d, int sink_blocks,
+                                int window_blocks, int block, float scale, flux_stream_t stream) {
+  if (!c || !q || !k_ring || !v_ring || !seqlens || !o)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: null tensor");
+  if (B < 1 || Hq < 1 || Hkv < 1 || sink_blocks < 0 || window_blocks < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: bad sizes");
+  if (d != 64 && d != 128)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_sa_compact: head_dim %d", d);
+  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_sa_compact: Hq/Hkv must be 1, 2 or 4");
+  if (block < 64 || block % 64 != 0)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_sa_compact: block must be a multiple of 64");
+  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: scale must be finite and positive");
+  if (static_cast<long long>(B) * Hkv > kMaxTickets)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_sa_compact: B * Hkv > %d", kMaxTickets);
+  if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: tensors must be 16-byte aligned");
+  const int rows = (sink_blocks + window_blocks) * block;
+  flux::DecodeLaunch p;
+  flux::decode_plan(B, Hkv, rows, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
+                    &p.chunk_fa, &p.chunk_sa);
+  const size_t nrow = static_cast<size_t>(B) * Hq * p.nsplit;
+  const size_t o_bytes = align256(nrow * d * sizeof(float));
+  if (o_bytes + align256(nrow * 2 * sizeof(float)) > c->workspace_bytes)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_sa_compact: workspace too small");
+  CUtensorMap tk, tv;
+  int rc;
+  if ((rc = make_map_4d(&tk, k_ring, d, Hkv, rows, B, 64, 64)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, v_ring, d, Hkv, rows, B, 64, 64)) != FLUX_OK) return rc;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.S_max = rows;
+  p.q = q;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.layer_mode = nullptr;
+  p.layer = 0;
+  p.sink_blocks = sink_blocks;
+  p.window_blocks = window_blocks;
+  p.block = block;
+  p.scale = scale;
+  p.part_o = static_cast<float*>(c->workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
+  p.tickets = c->tickets;
+  p.compact = 1;
+  p.st = status_of(c);
+  const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_sa_compact: launch");
 }
 
 }  // extern "C"
@@ -488,6 +566,7 @@ extern "C" int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cac
   p.part_ml = reinterpret_cast<float*>(dev->base + kNoAllocPartOff);
   p.part_o = reinterpret_cast<float*>(dev->base + kNoAllocPartOff + ml_bytes);
   p.tickets = tickets;
+  p.compact = 0;
   p.st = flux::DevStatus{err, 2000LL * 1000000LL};
   e = flux::launch_decode(tk, tv, p, s);
   if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: launch");

@@ -102,9 +102,9 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool fa = a.layer_mode == nullptr || a.layer_mode[a.layer] != 0;
+  const bool fa = !a.compact && (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
   int s = a.seqlens[b];
-  if (s < 0 || s > a.S_max) {
+  if (s < 0 || (!a.compact && s > a.S_max)) {
     if (i == 0 && g == 0 && tid == 0) raise_error(a.st.err, DEV_ERR_SEQLEN);
     s = 0;
   }
@@ -154,10 +154,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint8_t* kb = smem + st * L::STAGE;
         uint8_t* vb = kb + L::KT;
         mbar_arrive_expect_tx(&full[st], 2 * L::KT);
-        const int tok = rg.start + k * kTok;
+        int row = rg.start + k * kTok;
+        if (a.compact && row >= a.sink_blocks * a.block) {
+          // Ring slot of the token's block (a 64-token tile never straddles blocks).
+          const int j = row / a.block;
+          row = (a.sink_blocks + j % a.window_blocks) * a.block + row % a.block;
+        }
         for (int c = 0; c < L::CH; ++c) {
-          tma_load_4d(&tm_k, &full[st], kb + c * L::BOX, c * 64, g, tok, b);
-          tma_load_4d(&tm_v, &full[st], vb + c * L::BOX, c * 64, g, tok, b);
+          tma_load_4d(&tm_k, &full[st], kb + c * L::BOX, c * 64, g, row, b);
+          tma_load_4d(&tm_v, &full[st], vb + c * L::BOX, c * 64, g, row, b);
         }
         issued = k + 1;
       }

@@ -42,6 +42,7 @@ struct DecodeLaunch {
   int sink_blocks, window_blocks, block;
   float scale;
   int nsplit, chunk_fa, chunk_sa;
+  int compact;      // SA over the compact ring cache (sink + window blocks), S_max = ring rows
   float* part_o;    // [B, Hq, nsplit, d]
   float* part_ml;   // [B, Hq, nsplit, 2]
   int* tickets;     // [B, Hkv], zero between calls
@@ -72,6 +73,11 @@ struct RouteLaunch {
 };
 size_t route_workspace_bytes(int Hd, int H1);
 cudaError_t launch_route(const RouteLaunch& p, cudaStream_t stream);
+
+cudaError_t launch_ring_write(const uint16_t* k_src, const uint16_t* v_src, int n,
+                              const int32_t* seqlens, int B, int Hkv, int d, uint16_t* k_ring,
+                              uint16_t* v_ring, int sink, int window, int block, int* err,
+                              cudaStream_t stream);
 
 cudaError_t launch_streaming_mask(int nqb, int nkb, int sink, int window, uint8_t* mask,
                                   cudaStream_t stream);

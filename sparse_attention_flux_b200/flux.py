@@ -58,6 +58,9 @@ _SIGNATURES = {
                           _i, _f, _vp], _i),
     "flux_decode_workspace_bytes": ([_vp, _i, _i, _i, _i, _i, _i, _i, _i,
                                      ctypes.POINTER(ctypes.c_size_t)], _i),
+    "flux_kv_write": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _vp], _i),
+    "flux_attn_decode_sa_compact": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                     _f, _vp], _i),
     "flux_attn_decode_noalloc": ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i, _i,
                                   _i, _i, _f, _vp, _vp], _i),
 }
@@ -242,6 +245,42 @@ class Context:
                                       _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, d,
                                       _ptr(layer_mode), layer, sink_blocks, window_blocks, block,
                                       float(scale), _stream(stream)))
+
+    # ------------------------------------------------------------------ KV caches
+    def kv_write(self, k_src, v_src, seqlens, k_cache, v_cache, sink_blocks: int = 0,
+                 window_blocks: int = 0, block: int = 128, stream=None):
+        """Write the last n_src tokens of each sequence into a full cache (window_blocks=0)
+        or an SA layer's compact ring cache."""
+        import torch
+        for n_, t in (("k_src", k_src), ("v_src", v_src), ("k_cache", k_cache),
+                      ("v_cache", v_cache)):
+            _need(t, torch.bfloat16, n_, self.device)
+        _need(seqlens, torch.int32, "seqlens", self.device)
+        B, n_src, Hkv, d = k_src.shape
+        if v_src.shape != k_src.shape or k_cache.shape[0] != B or k_cache.shape[2:] != (Hkv, d) \
+                or v_cache.shape != k_cache.shape or seqlens.numel() < B:
+            raise ValueError("source / cache shapes are inconsistent")
+        _check(lib().flux_kv_write(self._h, _ptr(k_src), _ptr(v_src), n_src, _ptr(seqlens), B, Hkv,
+                                   d, _ptr(k_cache), _ptr(v_cache), k_cache.shape[1], sink_blocks,
+                                   window_blocks, block, _stream(stream)))
+
+    def attn_decode_sa_compact(self, q, k_ring, v_ring, seqlens, o, scale: float,
+                               sink_blocks: int = 1, window_blocks: int = 16, block: int = 128,
+                               lse=None, stream=None):
+        import torch
+        for n_, t in (("q", q), ("k_ring", k_ring), ("v_ring", v_ring), ("o", o)):
+            _need(t, torch.bfloat16, n_, self.device)
+        _need(seqlens, torch.int32, "seqlens", self.device)
+        _need(lse, torch.float32, "lse", self.device)
+        B, Hq, d = q.shape
+        rows = (sink_blocks + window_blocks) * block
+        if k_ring.shape[0] != B or k_ring.shape[1] != rows or k_ring.shape[3] != d \
+                or v_ring.shape != k_ring.shape or o.shape != q.shape:
+            raise ValueError("ring / q / o shapes are inconsistent")
+        _check(lib().flux_attn_decode_sa_compact(self._h, _ptr(q), _ptr(k_ring), _ptr(v_ring),
+                                                 _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq,
+                                                 k_ring.shape[2], d, sink_blocks, window_blocks,
+                                                 block, float(scale), _stream(stream)))
 
 
 def attn_decode_noalloc(q, k_cache, v_cache, seqlens, o, scale: float, layer_mode=None,
