@@ -13,7 +13,9 @@ needles per kv head):
 value = TFLOP/s over computed (query, key) pairs of both layers (4 d FLOPs per
 pair per head) / step time.  The decode half of the metric (KV GB/s) is timed
 in the same run on the 36-layer Qwen3-4B-shaped decode workload (batch 16, KV
-131072 + step, 18 FA / 18 SA layers, 64 steps) and reported under "decode".
+131072 + step, 18 FA / 18 SA layers, 64 steps; every layer appends the new token's
+K/V -- the full cache of an FA layer, the compact sink + window ring of an SA layer -- and
+decodes) and reported under "decode".
 
 Every input is seeded and synthetic; every timed input (640 MB for prefill,
 17 GB of KV for decode) is larger than the 126 MB L2, so no flush is needed.
@@ -234,47 +236,63 @@ class PrefillWorkload:
 
 
 class DecodeWorkload:
+    """36 layers, batch 16, KV 131072 + step.  Per layer and step the new token's K/V is
+    appended (flux_kv_write: the full cache of an FA layer, the compact ring of an SA
+    layer) and then decoded: FA layers read the whole cache, SA layers their ring of
+    sink + 16 blocks (the minimal KV the pages say SA layers keep)."""
+
     def __init__(self, ctx, seed, dev, steps):
         import torch
         from sparse_attention_flux_b200 import synth
         self.ctx, self.dev, self.steps = ctx, dev, steps
         self.S_max = DEC_S + steps
         shape = (DEC_B, self.S_max, HKV, D)
-        # 18 FA layers alias onto 2 physical caches (each 8.6 GB, far above L2);
-        # SA layers share one cache and touch only sink + window blocks.
+        # 18 FA layers alias onto 2 physical caches (each 8.6 GB, far above L2).
         self.fa_caches = [(synth.torch_normal_bf16(shape, seed + 10 * i + 1, dev),
                            synth.torch_normal_bf16(shape, seed + 10 * i + 2, dev)) for i in range(2)]
-        self.sa_cache = self.fa_caches[0]
         self.mode = torch.from_numpy(synth.layer_mode_choice(DEC_LAYERS, DEC_LAYERS // 2, seed)).to(dev)
         self.mode_h = self.mode.cpu().numpy()
+        ring = (DEC_B, (SINK + WIN) * BLOCK, HKV, D)
+        self.rings = {l: (synth.torch_normal_bf16(ring, seed + 1000 + 2 * l, dev),
+                          synth.torch_normal_bf16(ring, seed + 1001 + 2 * l, dev))
+                      for l in range(DEC_LAYERS) if not self.mode_h[l]}
         self.q = synth.torch_normal_bf16((DEC_B, HQ, D), seed + 99, dev)
+        self.new_k = synth.torch_normal_bf16((DEC_B, 1, HKV, D), seed + 97, dev)
+        self.new_v = synth.torch_normal_bf16((DEC_B, 1, HKV, D), seed + 98, dev)
         self.o = torch.empty_like(self.q)
-        self.seqlens = [torch.full((DEC_B,), DEC_S + s, dtype=torch.int32, device=dev)
+        self.seqlens = [torch.full((DEC_B,), DEC_S + s + 1, dtype=torch.int32, device=dev)
                         for s in range(steps)]
         self.scale = 1.0 / math.sqrt(D)
         kv_row = HKV * D * 2 * 2
-        self.bytes_fa = sum(DEC_B * (DEC_S + s) * kv_row for s in range(steps)) / steps
-        self.bytes_sa = sum(DEC_B * sa_decode_tokens(DEC_S + s, BLOCK, SINK, WIN) * kv_row
+        self.bytes_fa = sum(DEC_B * (DEC_S + s + 1) * kv_row for s in range(steps)) / steps
+        self.bytes_sa = sum(DEC_B * sa_decode_tokens(DEC_S + s + 1, BLOCK, SINK, WIN) * kv_row
                             for s in range(steps)) / steps
         n_fa = int(self.mode_h.sum())
         self.bytes_per_step = n_fa * self.bytes_fa + (DEC_LAYERS - n_fa) * self.bytes_sa
-        self.launches = DEC_LAYERS
+        self.launches = 2 * DEC_LAYERS
+        self.kv_gb = (2 * 2 * DEC_B * self.S_max * HKV * D * 2 +
+                      len(self.rings) * 2 * DEC_B * (SINK + WIN) * BLOCK * HKV * D * 2) / 1e9
 
     def step(self, s, fa_events=None):
         c = self.ctx
         fa_i = 0
+        sl = self.seqlens[s]
         for layer in range(DEC_LAYERS):
             if self.mode_h[layer]:
                 kc, vc = self.fa_caches[fa_i % 2]
                 fa_i += 1
+                timed = fa_events is not None and fa_i == 1
+                if timed:
+                    fa_events[0].record()
+                c.kv_write(self.new_k, self.new_v, sl, kc, vc)
+                c.attn_decode(self.q, kc, vc, sl, self.o, self.scale, layer_mode=self.mode,
+                              layer=layer, sink_blocks=SINK, window_blocks=WIN, block=BLOCK)
+                if timed:
+                    fa_events[1].record()
             else:
-                kc, vc = self.sa_cache
-            if fa_events is not None and self.mode_h[layer] and fa_i == 1:
-                fa_events[0].record()
-            c.attn_decode(self.q, kc, vc, self.seqlens[s], self.o, self.scale, layer_mode=self.mode,
-                          layer=layer, sink_blocks=SINK, window_blocks=WIN, block=BLOCK)
-            if fa_events is not None and self.mode_h[layer] and fa_i == 1:
-                fa_events[1].record()
+                kr, vr = self.rings[layer]
+                c.kv_write(self.new_k, self.new_v, sl, kr, vr, SINK, WIN, BLOCK)
+                c.attn_decode_sa_compact(self.q, kr, vr, sl, self.o, self.scale, SINK, WIN, BLOCK)
 
 
 def run_flux(args, rank, world, dev_index):
@@ -365,8 +383,9 @@ def run_flux(args, rank, world, dev_index):
         fa_dec_avg = statistics.mean(fa_dec_ms)
         fa_dec_gbs = dw.bytes_fa / (fa_dec_avg * 1e-3) / 1e9
         dec = {
-            "workload": "qwen3-4b-36L-routed-decode: B 16, KV 131072+step, 18 FA / 18 SA, "
-                        f"{dw.steps} steps",
+            "workload": "qwen3-4b-36L-routed-decode: B 16, KV 131072+step, 18 FA (full cache) / "
+                        f"18 SA (ring of sink 1 + 16 blocks), append + decode per layer, {dw.steps} steps",
+            "kv_resident_gb": round(dw.kv_gb, 2),
             "value": round(dec_gbs, 1), "unit": "GB/s (KV bytes that must be read)",
             "ms_per_step": round(dec_ms, 4), "gpu_launches_per_step": dw.launches,
             "frac_of_hbm": round(dec_gbs / peaks["hbm_gbs"], 4),
@@ -375,7 +394,7 @@ def run_flux(args, rank, world, dev_index):
         }
         roof_dec = {"bound": "hbm", "achieved": round(fa_dec_gbs, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4),
-                    "traffic": None, "kernel": "decode_kernel<128,4> (FA layer)"}
+                    "traffic": None, "kernel": "decode_kernel<128,4> (FA layer, incl. its append)"}
         dec["roofline"] = roof_dec
         del dw
     ctx.close()

@@ -13,6 +13,7 @@
  *   flux_build_streaming_mask  sink + window block mask     -> mask[nqb][nkb]
  *   flux_build_block_index     block mask                   -> CSR row_ptr/col
  *   flux_attn_prefill          one layer, FA or SA per layer_mode[layer]
+ *   flux_attn_prefill_soft     r FA + (1 - r) SA, the training-time soft routing
  *   flux_attn_decode           one layer, one new token per sequence
  *   flux_kv_write              append / fill a full cache or an SA layer's ring
  *   flux_attn_decode_sa_compact  SA decode over the ring (sink + last W blocks)
@@ -151,6 +152,19 @@ int flux_attn_prefill(flux_ctx* ctx, const uint16_t* q, const uint16_t* k, const
                       const uint8_t* layer_mode, int layer,
                       const int32_t* row_ptr, const int32_t* col, int nqb, int block,
                       float scale, flux_stream_t stream);
+
+/* Soft-routing forward blend (gist.science summary section 2, "training
+ * process": during training the continuous router weight r_soft combines the
+ * two paths, o = r FA + (1 - r) SA).  Forward only: runs the FA pass into o,
+ * then the SA pass (over the CSR list), whose epilogue reads that row of o and
+ * writes r * o_FA + (1 - r) * o_SA with r = score[layer] read on the device
+ * (the `score` output of flux_route).  Shapes, layouts and limits as
+ * flux_attn_prefill; no lse.  r = 1 gives FA's output exactly, r = 0 SA's. */
+int flux_attn_prefill_soft(flux_ctx* ctx, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           uint16_t* o, int B, int T, int Hq, int Hkv, int d,
+                           const float* score, int layer,
+                           const int32_t* row_ptr, const int32_t* col, int nqb, int block,
+                           float scale, flux_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * Decode attention for one layer and one new token per sequence (gist.science

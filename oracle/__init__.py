@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
             L.oracle_block_index.argtypes = [_u8p, i, i, _i32p, _i32p]
             L.oracle_attn_prefill.argtypes = [_u16p, _u16p, _u16p, i, i, i, i, i, _vp, i, i, d,
                                               _vp, ctypes.c_longlong, _f64p, _vp]
+            L.oracle_attn_prefill_soft.argtypes = [_u16p, _u16p, _u16p, i, i, i, i, i, _u8p, i, i, d,
+                                                   d, _vp, ctypes.c_longlong, _f64p]
             L.oracle_attn_probs.argtypes = [_u16p, _u16p, i, i, i, i, i, _vp, i, i, d, i, i, _f64p]
             L.oracle_attn_decode.argtypes = [_u16p, _u16p, _u16p, i, _i32p, i, i, i, i, i, i, i,
                                              i, d, _f64p, _vp]
@@ -182,6 +184,25 @@ def attn_prefill(q, k, v, scale: float, block_mask=None, block: int = 0, rows=No
     if rows is None:
         return o.reshape(B, T, Hq, d), lse.reshape(B, T, Hq)
     return o, lse
+
+
+def attn_prefill_soft(q, k, v, scale: float, r: float, block_mask, block: int, rows=None):
+    """Soft-routing blend r * FA + (1 - r) * SA in fp64; shapes as attn_prefill."""
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    mask = np.ascontiguousarray(block_mask, np.uint8)
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, np.int32).reshape(-1, 3)
+        n = rows.shape[0]
+    else:
+        n = B * T * Hq
+    o = np.empty((n, d), np.float64)
+    _check(lib().oracle_attn_prefill_soft(q, k, v, B, T, Hq, Hkv, d, mask, mask.shape[1], block,
+                                          scale, r, _ptr(rows), n, o), "attn_prefill_soft")
+    return o if rows is not None else o.reshape(B, T, Hq, d)
 
 
 def attn_probs(q, k, scale: float, b: int, h: int, block_mask=None, block: int = 0):

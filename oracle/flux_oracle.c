@@ -287,6 +287,31 @@ int oracle_attn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v,
     return bad ? -1 : 0;
 }
 
+/* Soft routing, forward only (gist.science summary, section 2, "training
+ * process": the continuous weight r_soft forms the convex combination of the
+ * FA and SA outputs).  o = r * FA + (1 - r) * SA, row by row, with the SA
+ * block mask given.  rows as in oracle_attn_prefill. */
+int oracle_attn_prefill_soft(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             int B, int T, int Hq, int Hkv, int d,
+                             const uint8_t* block_mask, int nkb, int block, double scale, double r,
+                             const int32_t* rows, long long n_rows, double* o) {
+    if (!block_mask) return -1;
+    long long total = rows ? n_rows : (long long)B * T * Hq;
+    double* o_fa = (double*)malloc(sizeof(double) * (size_t)total * d);
+    double* o_sa = (double*)malloc(sizeof(double) * (size_t)total * d);
+    int rc = -1;
+    if (o_fa && o_sa &&
+        oracle_attn_prefill(q, k, v, B, T, Hq, Hkv, d, NULL, 0, 0, scale, rows, n_rows, o_fa, NULL) == 0 &&
+        oracle_attn_prefill(q, k, v, B, T, Hq, Hkv, d, block_mask, nkb, block, scale, rows, n_rows,
+                            o_sa, NULL) == 0) {
+        for (long long i = 0; i < total * d; ++i) o[i] = r * o_fa[i] + (1.0 - r) * o_sa[i];
+        rc = 0;
+    }
+    free(o_fa);
+    free(o_sa);
+    return rc;
+}
+
 /* The full probability matrix P[t][u] of one (b, h) pair, T x T, for the
  * invariant checks (rows sum to one, masked and causal entries are zero). */
 int oracle_attn_probs(const uint16_t* q, const uint16_t* k, int B, int T, int Hq, int Hkv, int d,

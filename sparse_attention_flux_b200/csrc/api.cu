@@ -288,9 +288,53 @@ int flux_attn_prefill(flux_ctx* c, const uint16_t* q, const uint16_t* k, const u
   p.col = col;
   p.o = o;
   p.lse = lse;
+  p.force_mode = -1;
+  p.blend_score = nullptr;
   p.st = status_of(c);
   const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill: launch");
+}
+
+int flux_attn_prefill_soft(flux_ctx* c, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           uint16_t* o, int B, int T, int Hq, int Hkv, int d, const float* score,
+                           int layer, const int32_t* row_ptr, const int32_t* col, int nqb,
+                           int block, float scale, flux_stream_t stream) {
+  if (!score || layer < 0)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_soft: score and a layer are required");
+  if (!row_ptr || !col)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_soft: row_ptr/col are required");
+  if (block > 0 && T > 0 && nqb < (T + block - 1) / block)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_soft: nqb %d < ceil(T / block)", nqb);
+  if (T > 0 && (T + 127) / 128 > flux::kPrefillMaxKvTiles)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_soft: T <= %d", flux::kPrefillMaxKvTiles * 128);
+  // Argument checks and tensor maps exactly as flux_attn_prefill (FA pass first).
+  int rc = flux_attn_prefill(c, q, k, v, o, nullptr, B, T, Hq, Hkv, d, nullptr, 0, row_ptr, col,
+                             nqb, block, scale, stream);
+  if (rc != FLUX_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  flux::PrefillLaunch p;
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.block = block;
+  p.nqb = nqb;
+  p.scale = scale;
+  p.layer_mode = nullptr;
+  p.layer = layer;
+  p.row_ptr = row_ptr;
+  p.col = col;
+  p.o = o;
+  p.lse = nullptr;
+  p.force_mode = 0;          // the SA pass, blended into the FA output in its epilogue
+  p.blend_score = score;
+  p.st = status_of(c);
+  const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill_soft: launch");
 }
 
 int flux_decode_workspace_bytes(flux_ctx* c, int B, int Hq, int Hkv, int d, int S_max,

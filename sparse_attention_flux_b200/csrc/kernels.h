@@ -25,6 +25,8 @@ struct PrefillLaunch {
   const int32_t* col;
   uint16_t* o;
   float* lse;
+  int force_mode;            // -1: layer_mode decides; 0: SA; 1: FA
+  const float* blend_score;  // non-null: o = r * o + (1 - r) * this pass, r = blend_score[layer]
   DevStatus st;
 };
 int prefill_smem_bytes(int d);

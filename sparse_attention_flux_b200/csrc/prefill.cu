@@ -52,6 +52,8 @@ struct PrefillArgs {
   const int32_t* col;
   uint16_t* o;
   float* lse;
+  int force_mode;            // -1: read layer_mode; 0: SA; 1: FA
+  const float* blend_score;  // soft routing: o = r * o(previous) + (1 - r) * this, r = score[layer]
   DevStatus st;
 };
 
@@ -150,7 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pair = a.npair - 1 - static_cast<int>(blockIdx.x) / per_pair;
   const int rem = static_cast<int>(blockIdx.x) % per_pair;
   const int b = rem / a.Hq, h = rem % a.Hq, g = h / a.G;
-  const bool fa = a.layer_mode == nullptr || a.layer_mode[a.layer] != 0;
+  const bool fa = a.force_mode >= 0 ? a.force_mode == 1
+                                    : (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
   const int q0 = pair * 256;
 
   if (threadIdx.x == 0) {
@@ -374,6 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (n > 0 && ok && mbar_wait(&bars[B_OD], 0, a.st)) {
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      // Soft routing: blend with the row already in o (the other path's output).
+      const float r = a.blend_score ? a.blend_score[a.layer] : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -381,13 +386,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(a.o + row_elem + c * 32);
+          if (a.blend_score) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 prev = dst[u];
+              const uint32_t pw[4] = {prev.x, prev.y, prev.z, prev.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                v[u * 8 + 2 * e] = __float_as_uint(
+                    fmaf(r, bf16lo_to_f32(pw[e]), (1.f - r) * __uint_as_float(v[u * 8 + 2 * e]) * inv));
+                v[u * 8 + 2 * e + 1] = __float_as_uint(
+                    fmaf(r, bf16hi_to_f32(pw[e]), (1.f - r) * __uint_as_float(v[u * 8 + 2 * e + 1]) * inv));
+              }
+            }
+          }
+          const float sc = a.blend_score ? 1.f : inv;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[u * 8 + 0]) * inv, __uint_as_float(v[u * 8 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(v[u * 8 + 2]) * inv, __uint_as_float(v[u * 8 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(v[u * 8 + 4]) * inv, __uint_as_float(v[u * 8 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(v[u * 8 + 6]) * inv, __uint_as_float(v[u * 8 + 7]) * inv);
+            w.x = pack_bf16x2(__uint_as_float(v[u * 8 + 0]) * sc, __uint_as_float(v[u * 8 + 1]) * sc);
+            w.y = pack_bf16x2(__uint_as_float(v[u * 8 + 2]) * sc, __uint_as_float(v[u * 8 + 3]) * sc);
+            w.z = pack_bf16x2(__uint_as_float(v[u * 8 + 4]) * sc, __uint_as_float(v[u * 8 + 5]) * sc);
+            w.w = pack_bf16x2(__uint_as_float(v[u * 8 + 6]) * sc, __uint_as_float(v[u * 8 + 7]) * sc);
             dst[u] = w;
           }
         }
@@ -397,9 +417,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       }
     } else if (valid) {
-      // No visible key (or an aborted tile): the row's output is zero.
+      // No visible key (or an aborted tile): this pass contributes zero.
       uint4* dst = reinterpret_cast<uint4*>(a.o + row_elem);
-      for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0, 0, 0, 0);
+      const float r = a.blend_score ? a.blend_score[a.layer] : 0.f;
+      for (int u = 0; u < D / 8; ++u) {
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (a.blend_score) {
+          const uint4 prev = dst[u];
+          w.x = pack_bf16x2(r * bf16lo_to_f32(prev.x), r * bf16hi_to_f32(prev.x));
+          w.y = pack_bf16x2(r * bf16lo_to_f32(prev.y), r * bf16hi_to_f32(prev.y));
+          w.z = pack_bf16x2(r * bf16lo_to_f32(prev.z), r * bf16hi_to_f32(prev.z));
+          w.w = pack_bf16x2(r * bf16lo_to_f32(prev.w), r * bf16hi_to_f32(prev.w));
+        }
+        dst[u] = w;
+      }
       if (a.lse) a.lse[(static_cast<size_t>(b) * a.Hq + h) * a.T + t_row] = -INFINITY;
     }
   }
@@ -434,6 +465,8 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   a.col = p.col;
   a.o = p.o;
   a.lse = p.lse;
+  a.force_mode = p.force_mode;
+  a.blend_score = p.blend_score;
   a.st = p.st;
   const dim3 grid(static_cast<unsigned>(a.npair) * p.Hq * p.B);
   if (p.d == 64) {

@@ -58,6 +58,8 @@ _SIGNATURES = {
                           _i, _f, _vp], _i),
     "flux_decode_workspace_bytes": ([_vp, _i, _i, _i, _i, _i, _i, _i, _i,
                                      ctypes.POINTER(ctypes.c_size_t)], _i),
+    "flux_attn_prefill_soft": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _i,
+                                _i, _f, _vp], _i),
     "flux_kv_write": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "flux_attn_decode_sa_compact": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                      _f, _vp], _i),
@@ -223,6 +225,24 @@ class Context:
         _check(lib().flux_attn_prefill(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
                                        T, Hq, Hkv, d, _ptr(layer_mode), layer, _ptr(row_ptr),
                                        _ptr(col), nqb, block, float(scale), _stream(stream)))
+
+    def attn_prefill_soft(self, q, k, v, o, scale: float, score, layer: int, row_ptr, col,
+                          block: int = 128, stream=None):
+        """o = r * FA + (1 - r) * SA with r = score[layer] (device), forward only."""
+        import torch
+        for n_, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+            _need(t, torch.bfloat16, n_, self.device)
+        _need(score, torch.float32, "score", self.device)
+        _need(row_ptr, torch.int32, "row_ptr", self.device)
+        _need(col, torch.int32, "col", self.device)
+        B, T, Hq, d = q.shape
+        Hkv = k.shape[2]
+        if k.shape != (B, T, Hkv, d) or v.shape != k.shape or o.shape != q.shape:
+            raise ValueError("q/k/v/o shapes are inconsistent")
+        _check(lib().flux_attn_prefill_soft(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, T, Hq,
+                                            Hkv, d, _ptr(score), layer, _ptr(row_ptr), _ptr(col),
+                                            row_ptr.numel() - 1, block, float(scale),
+                                            _stream(stream)))
 
     def attn_decode(self, q, k_cache, v_cache, seqlens, o, scale: float, layer_mode=None,
                     layer: int = 0, sink_blocks: int = 1, window_blocks: int = 16,

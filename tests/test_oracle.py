@@ -332,3 +332,18 @@ def test_needle_query_concentrates_on_needles():
     for i, (h, r, pos) in enumerate(needles):
         target = V[0, pos, h // (Hq // Hkv)].mean(0)
         assert np.abs(o[i] - target).max() < 0.05
+
+
+def test_soft_blend_reduces_to_fa_and_sa_and_is_convex():
+    # r = 1 and r = 0 give FA and SA exactly; any r lies on the segment between them.
+    B, T, Hq, Hkv, d, block = 1, 160, 2, 1, 16, 32
+    q, k, v = synth.attention_inputs(B, T, Hq, Hkv, d, seed=61)
+    m = oracle.streaming_mask(5, 5, 1, 2)
+    fa, _ = oracle.attn_prefill(q, k, v, 0.25)
+    sa, _ = oracle.attn_prefill(q, k, v, 0.25, block_mask=m, block=block)
+    assert np.array_equal(oracle.attn_prefill_soft(q, k, v, 0.25, 1.0, m, block), fa)
+    assert np.array_equal(oracle.attn_prefill_soft(q, k, v, 0.25, 0.0, m, block), sa)
+    mid = oracle.attn_prefill_soft(q, k, v, 0.25, 0.3, m, block)
+    np.testing.assert_allclose(mid, 0.3 * fa + 0.7 * sa, rtol=0, atol=1e-15)
+    # rows where the SA mask keeps every key (the first W blocks) are unchanged by r
+    np.testing.assert_allclose(mid[0, :64], fa[0, :64], rtol=0, atol=1e-15)
