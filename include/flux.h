@@ -227,6 +227,30 @@ int flux_attn_decode_sa_compact(flux_ctx* ctx, const uint16_t* q, const uint16_t
                                 flux_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Per-head routing (the contrast case).  Flux Attention routes whole layers;
+ * the head-level alternative it is compared with (Elastic Attention on the
+ * same page list) routes each attention head, and the arXiv abstract states
+ * that head-level dynamic sparsity causes load imbalance and synchronisation
+ * long-tails in decoding.  These two calls make that measurable:
+ *   head_mode [Hq] uint8 device array: 1 = FA, 0 = SA for query head h.
+ * flux_attn_prefill_heads: as flux_attn_prefill, mode per query head.
+ * flux_attn_decode_heads: as flux_attn_decode; the CTA serving a GQA group
+ * streams the whole history if any head of the group is FA, and masks the
+ * tokens outside the sink + window blocks for its SA heads -- so a mixed group
+ * costs a full FA read.  Results equal per-head FA / SA attention. */
+int flux_attn_prefill_heads(flux_ctx* ctx, const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, uint16_t* o, float* lse, int B, int T,
+                            int Hq, int Hkv, int d, const uint8_t* head_mode,
+                            const int32_t* row_ptr, const int32_t* col, int nqb, int block,
+                            float scale, flux_stream_t stream);
+
+int flux_attn_decode_heads(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_cache,
+                           const uint16_t* v_cache, int S_max, const int32_t* seqlens,
+                           uint16_t* o, float* lse, int B, int Hq, int Hkv, int d,
+                           const uint8_t* head_mode, int sink_blocks, int window_blocks,
+                           int block, float scale, flux_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * Decode attention that allocates nothing.  The pages have no counterpart of
  * this entry point; it exists for callers that cannot call cudaMalloc: an
  * inference engine that reserves all device memory up front and owns every

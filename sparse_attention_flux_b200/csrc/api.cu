@@ -289,6 +289,7 @@ int flux_attn_prefill(flux_ctx* c, const uint16_t* q, const uint16_t* k, const u
   p.o = o;
   p.lse = lse;
   p.force_mode = -1;
+  p.head_mode = nullptr;
   p.blend_score = nullptr;
   p.st = status_of(c);
   const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
@@ -331,6 +332,7 @@ int flux_attn_prefill_soft(flux_ctx* c, const uint16_t* q, const uint16_t* k, co
   p.o = o;
   p.lse = nullptr;
   p.force_mode = 0;          // the SA pass, blended into the FA output in its epilogue
+  p.head_mode = nullptr;
   p.blend_score = score;
   p.st = status_of(c);
   const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
@@ -403,6 +405,7 @@ int flux_attn_decode(flux_ctx* c, const uint16_t* q, const uint16_t* k_cache,
   p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
   p.tickets = c->tickets;
   p.compact = 0;
+  p.head_mode = nullptr;
   p.st = status_of(c);
   const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode: launch");
@@ -480,6 +483,7 @@ int flux_attn_decode_sa_compact(flux_ctx* c, const uint16_t* q, const uint16_t* 
   p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
   p.tickets = c->tickets;
   p.compact = 1;
+  p.head_mode = nullptr;
   p.st = status_of(c);
   const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_sa_compact: launch");
@@ -611,6 +615,7 @@ extern "C" int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cac
   p.part_o = reinterpret_cast<float*>(dev->base + kNoAllocPartOff + ml_bytes);
   p.tickets = tickets;
   p.compact = 0;
+  p.head_mode = nullptr;
   p.st = flux::DevStatus{err, 2000LL * 1000000LL};
   e = flux::launch_decode(tk, tv, p, s);
   if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: launch");
@@ -618,4 +623,116 @@ extern "C" int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cac
                     cudaSuccess)
     return cuda_fail(e, "flux_attn_decode_noalloc: copy status");
   return FLUX_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Per-head routing: the contrast case for layer-level routing.
+
+extern "C" int flux_attn_prefill_heads(flux_ctx* c, const uint16_t* q, const uint16_t* k,
+                                       const uint16_t* v, uint16_t* o, float* lse, int B, int T,
+                                       int Hq, int Hkv, int d, const uint8_t* head_mode,
+                                       const int32_t* row_ptr, const int32_t* col, int nqb,
+                                       int block, float scale, flux_stream_t stream) {
+  if (!head_mode) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: head_mode is required");
+  if (!row_ptr || !col)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: row_ptr/col are required");
+  if (block > 0 && T > 0 && nqb < (T + block - 1) / block)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_heads: nqb %d < ceil(T / block)", nqb);
+  if (T > 0 && (T + 127) / 128 > flux::kPrefillMaxKvTiles)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_heads: T <= %d", flux::kPrefillMaxKvTiles * 128);
+  // Same checks as flux_attn_prefill (run with layer_mode absent, then relaunched per head).
+  if (!c || !q || !k || !v || !o) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: null tensor");
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_heads: sizes must be positive");
+  if (d != 64 && d != 128) return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill_heads: head_dim %d", d);
+  if (Hq % Hkv != 0) return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill_heads: Hq %% Hkv != 0");
+  if (block != 64 && (block < 128 || block % 128 != 0))
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill_heads: block %d", block);
+  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: scale must be finite and positive");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: tensors must be 16-byte aligned");
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  flux::PrefillLaunch p;
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.block = block;
+  p.nqb = nqb;
+  p.scale = scale;
+  p.layer_mode = nullptr;
+  p.layer = 0;
+  p.row_ptr = row_ptr;
+  p.col = col;
+  p.o = o;
+  p.lse = lse;
+  p.force_mode = -1;
+  p.head_mode = head_mode;
+  p.blend_score = nullptr;
+  p.st = status_of(c);
+  const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill_heads: launch");
+}
+
+extern "C" int flux_attn_decode_heads(flux_ctx* c, const uint16_t* q, const uint16_t* k_cache,
+                                      const uint16_t* v_cache, int S_max, const int32_t* seqlens,
+                                      uint16_t* o, float* lse, int B, int Hq, int Hkv, int d,
+                                      const uint8_t* head_mode, int sink_blocks, int window_blocks,
+                                      int block, float scale, flux_stream_t stream) {
+  if (!head_mode) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: head_mode is required");
+  if (!c || !q || !k_cache || !v_cache || !seqlens || !o)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: null tensor");
+  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_heads: sizes must be positive");
+  if (d != 64 && d != 128) return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_heads: head_dim %d", d);
+  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_heads: Hq/Hkv must be 1, 2 or 4");
+  if (block < 1 || sink_blocks < 0 || window_blocks < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: bad block / sink / window");
+  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: scale must be finite and positive");
+  if (static_cast<long long>(B) * Hkv > kMaxTickets)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_heads: B * Hkv > %d", kMaxTickets);
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: tensors must be 16-byte aligned");
+  flux::DecodeLaunch p;
+  flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
+                    &p.chunk_fa, &p.chunk_sa);
+  const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
+  const size_t o_bytes = align256(rows * d * sizeof(float));
+  if (o_bytes + align256(rows * 2 * sizeof(float)) > c->workspace_bytes)
+    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_heads: workspace too small");
+  CUtensorMap tk, tv;
+  int rc;
+  if ((rc = make_map_4d(&tk, k_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, v_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.S_max = S_max;
+  p.q = q;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.layer_mode = nullptr;
+  p.layer = 0;
+  p.sink_blocks = sink_blocks;
+  p.window_blocks = window_blocks;
+  p.block = block;
+  p.scale = scale;
+  p.part_o = static_cast<float*>(c->workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
+  p.tickets = c->tickets;
+  p.compact = 0;
+  p.head_mode = head_mode;
+  p.st = status_of(c);
+  const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_heads: launch");
 }

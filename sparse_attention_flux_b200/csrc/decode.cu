@@ -102,7 +102,17 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool fa = !a.compact && (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
+  // Per-head routing: the group reads the FA range if any of its heads is FA;
+  // its SA heads then mask every token outside the sink + window blocks.
+  const uint8_t* hm = a.head_mode ? a.head_mode + g * G : nullptr;
+  bool fa;
+  if (hm) {
+    fa = false;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) fa |= hm[hh] != 0;
+  } else {
+    fa = !a.compact && (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
+  }
   int s = a.seqlens[b];
   if (s < 0 || (!a.compact && s > a.S_max)) {
     if (i == 0 && g == 0 && tid == 0) raise_error(a.st.err, DEV_ERR_SEQLEN);
@@ -190,6 +200,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const float sl2 = a.scale * 1.4426950408889634f;
     const int mrow = lane & 7, msel = lane >> 3;     // ldmatrix row and matrix index
+    const bool row_sa = fa && hm != nullptr && gq < G && hm[gq] == 0;
+    const int nbs = (s + a.block - 1) / a.block;
     const int wtok = warp * 16;
     for (int k = 0; k < ntiles; ++k) {
       const int st = k % kStages;
@@ -217,7 +229,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int n = 0; n < 2; ++n)
 #pragma unroll
         for (int e = 0; e < 2; ++e)
-          x[n * 2 + e] = (gq < G && tok0 + 8 * n + e < rg.end) ? sc[n][e] : -INFINITY;
+        {
+          const int u = tok0 + 8 * n + e;
+          const bool keep = gq < G && u < rg.end &&
+                            (!row_sa || u / a.block < a.sink_blocks ||
+                             u / a.block >= nbs - a.window_blocks);
+          x[n * 2 + e] = keep ? sc[n][e] : -INFINITY;
+        }
       float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
       mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));

@@ -26,6 +26,7 @@ struct PrefillLaunch {
   uint16_t* o;
   float* lse;
   int force_mode;            // -1: layer_mode decides; 0: SA; 1: FA
+  const uint8_t* head_mode;  // per-query-head routing [Hq], overrides layer_mode
   const float* blend_score;  // non-null: o = r * o + (1 - r) * this pass, r = blend_score[layer]
   DevStatus st;
 };
@@ -45,6 +46,7 @@ struct DecodeLaunch {
   float scale;
   int nsplit, chunk_fa, chunk_sa;
   int compact;      // SA over the compact ring cache (sink + window blocks), S_max = ring rows
+  const uint8_t* head_mode;  // per-query-head routing [Hq] (overrides layer_mode), or null
   float* part_o;    // [B, Hq, nsplit, d]
   float* part_ml;   // [B, Hq, nsplit, 2]
   int* tickets;     // [B, Hkv], zero between calls

@@ -53,6 +53,7 @@ struct PrefillArgs {
   uint16_t* o;
   float* lse;
   int force_mode;            // -1: read layer_mode; 0: SA; 1: FA
+  const uint8_t* head_mode;  // per-query-head routing [Hq] (overrides layer_mode), or null
   const float* blend_score;  // soft routing: o = r * o(previous) + (1 - r) * this, r = score[layer]
   DevStatus st;
 };
@@ -153,7 +154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rem = static_cast<int>(blockIdx.x) % per_pair;
   const int b = rem / a.Hq, h = rem % a.Hq, g = h / a.G;
   const bool fa = a.force_mode >= 0 ? a.force_mode == 1
-                                    : (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
+                 : a.head_mode     ? a.head_mode[h] != 0
+                                   : (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
   const int q0 = pair * 256;
 
   if (threadIdx.x == 0) {
@@ -466,6 +468,7 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   a.o = p.o;
   a.lse = p.lse;
   a.force_mode = p.force_mode;
+  a.head_mode = p.head_mode;
   a.blend_score = p.blend_score;
   a.st = p.st;
   const dim3 grid(static_cast<unsigned>(a.npair) * p.Hq * p.B);

@@ -60,6 +60,10 @@ _SIGNATURES = {
                                      ctypes.POINTER(ctypes.c_size_t)], _i),
     "flux_attn_prefill_soft": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _i,
                                 _i, _f, _vp], _i),
+    "flux_attn_prefill_heads": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp,
+                                 _i, _i, _f, _vp], _i),
+    "flux_attn_decode_heads": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i, _i,
+                                _i, _f, _vp], _i),
     "flux_kv_write": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "flux_attn_decode_sa_compact": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                      _f, _vp], _i),
@@ -265,6 +269,41 @@ class Context:
                                       _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, d,
                                       _ptr(layer_mode), layer, sink_blocks, window_blocks, block,
                                       float(scale), _stream(stream)))
+
+    # ------------------------------------------------------------------ per-head routing
+    def attn_prefill_heads(self, q, k, v, o, scale: float, head_mode, row_ptr, col,
+                           block: int = 128, lse=None, stream=None):
+        import torch
+        for n_, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+            _need(t, torch.bfloat16, n_, self.device)
+        _need(head_mode, torch.uint8, "head_mode", self.device)
+        _need(lse, torch.float32, "lse", self.device)
+        B, T, Hq, d = q.shape
+        Hkv = k.shape[2]
+        if head_mode.numel() < Hq or k.shape != (B, T, Hkv, d) or v.shape != k.shape:
+            raise ValueError("shapes are inconsistent")
+        _check(lib().flux_attn_prefill_heads(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                             B, T, Hq, Hkv, d, _ptr(head_mode), _ptr(row_ptr),
+                                             _ptr(col), row_ptr.numel() - 1, block, float(scale),
+                                             _stream(stream)))
+
+    def attn_decode_heads(self, q, k_cache, v_cache, seqlens, o, scale: float, head_mode,
+                          sink_blocks: int = 1, window_blocks: int = 16, block: int = 128,
+                          lse=None, stream=None):
+        import torch
+        for n_, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("o", o)):
+            _need(t, torch.bfloat16, n_, self.device)
+        _need(head_mode, torch.uint8, "head_mode", self.device)
+        _need(seqlens, torch.int32, "seqlens", self.device)
+        _need(lse, torch.float32, "lse", self.device)
+        B, Hq, d = q.shape
+        _, S_max, Hkv, _ = k_cache.shape
+        if head_mode.numel() < Hq or v_cache.shape != k_cache.shape:
+            raise ValueError("shapes are inconsistent")
+        _check(lib().flux_attn_decode_heads(self._h, _ptr(q), _ptr(k_cache), _ptr(v_cache), S_max,
+                                            _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, d,
+                                            _ptr(head_mode), sink_blocks, window_blocks, block,
+                                            float(scale), _stream(stream)))
 
     # ------------------------------------------------------------------ KV caches
     def kv_write(self, k_src, v_src, seqlens, k_cache, v_cache, sink_blocks: int = 0,
