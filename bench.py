@@ -273,6 +273,44 @@ class DecodeWorkload:
         self.kv_gb = (2 * 2 * DEC_B * self.S_max * HKV * D * 2 +
                       len(self.rings) * 2 * DEC_B * (SINK + WIN) * BLOCK * HKV * D * 2) / 1e9
 
+    def granularity(self, steps):
+        """ms per 36-layer decode step, layer-level vs head-level routing at the same SA
+        fraction (one half): layer level routes 18 whole layers to SA; head level routes a
+        seeded half of each layer's query heads to SA, so a GQA group containing any FA
+        head streams the full history (no appends; full caches for every layer)."""
+        import torch
+        from sparse_attention_flux_b200 import synth
+        rng = synth.rng(4242)
+        heads = [torch.from_numpy((rng.permutation(HQ) < HQ // 2).astype(np.uint8)).to(self.dev)
+                 for _ in range(DEC_LAYERS)]
+        sl = self.seqlens[0]
+        out = {}
+        for level in ("layer", "head"):
+            def one():
+                for layer in range(DEC_LAYERS):
+                    kc, vc = self.fa_caches[layer % 2]
+                    if level == "layer":
+                        self.ctx.attn_decode(self.q, kc, vc, sl, self.o, self.scale,
+                                             layer_mode=self.mode, layer=layer, sink_blocks=SINK,
+                                             window_blocks=WIN, block=BLOCK)
+                    else:
+                        self.ctx.attn_decode_heads(self.q, kc, vc, sl, self.o, self.scale,
+                                                   heads[layer], SINK, WIN, BLOCK)
+            one()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(steps):
+                one()
+            b.record()
+            b.synchronize()
+            out[level + "_ms_per_step"] = round(a.elapsed_time(b) / steps, 4)
+        frac_groups_all_sa = float(np.mean([(h.cpu().numpy().reshape(HKV, HQ // HKV) == 0).all(1).mean()
+                                            for h in heads]))
+        out["head_over_layer"] = round(out["head_ms_per_step"] / out["layer_ms_per_step"], 3)
+        out["groups_fully_sa_at_head_level"] = round(frac_groups_all_sa, 3)
+        out["sa_fraction"] = 0.5
+        return out
+
     def step(self, s, fa_events=None):
         c = self.ctx
         fa_i = 0
@@ -351,6 +389,21 @@ def run_flux(args, rank, world, dev_index):
     e2e_ms = ranks_max(s0.elapsed_time(s1) / e2e_steps)
     e2e_value = whole_job_rate(wl.flops, world, e2e_ms)
 
+    # soft-routing forward blend on the same layer: FA pass + SA pass with a blend epilogue
+    score = torch.tensor([0.3], dtype=torch.float32, device=dev)
+    soft = lambda: ctx.attn_prefill_soft(wl.q, wl.k, wl.v, wl.o[0], wl.scale, score, 0,
+                                         wl.row_ptr, wl.col, BLOCK)
+    soft()
+    s0, s1 = new_ev(), new_ev()
+    s0.record()
+    for _ in range(3):
+        soft()
+    s1.record()
+    s1.synchronize()
+    soft_ms = s0.elapsed_time(s1) / 3
+    soft_line = {"ms": round(soft_ms, 4), "TFLOP/s": round(wl.flops / (soft_ms * 1e-3) / 1e12, 1),
+                 "note": "flux_attn_prefill_soft, r = 0.3: FA + SA passes, blended in the SA epilogue"}
+
     h2d_bytes, d2h_bytes, launches = wl.h2d_bytes, wl.d2h_bytes, wl.launches * args.steps
     fa_avg = statistics.mean(fa_ms)
     sa_avg = statistics.mean(sa_ms)
@@ -396,6 +449,8 @@ def run_flux(args, rank, world, dev_index):
                     "unit": "GB/s", "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4),
                     "traffic": None, "kernel": "decode_kernel<128,4> (FA layer, incl. its append)"}
         dec["roofline"] = roof_dec
+        dec["routing_granularity"] = dw.granularity(8)
+        ctx.check()
         del dw
     ctx.close()
 
@@ -416,6 +471,7 @@ def run_flux(args, rank, world, dev_index):
         "sa_prefill": {"TFLOP/s": round(sa_tflops, 1), "ms": round(sa_avg, 4),
                        "frac": round(sa_tflops / peak_t, 4)},
         "fa_prefill": {"TFLOP/s": round(fa_tflops, 1), "ms": round(fa_avg, 4)},
+        "soft_prefill": soft_line,
         "decode": dec,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
