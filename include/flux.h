@@ -85,6 +85,16 @@ int flux_ctx_check(flux_ctx* ctx, flux_stream_t stream);
  * release its resources and return. */
 int flux_ctx_set_spin_limit_ms(flux_ctx* ctx, int ms);
 
+/* Self-test of the failure path every pipeline kernel relies on: launches one
+ * thread that waits on an mbarrier nothing ever arrives at, through the same
+ * bounded wait (here limited to spin_limit_ms, 1..10000).  The wait gives up,
+ * records the timeout in the device error word and the kernel returns; a
+ * following flux_ctx_check returns FLUX_ERR_TIMEOUT and clears the word, and
+ * the context stays usable.  waited_us (device int, optional) receives the
+ * time the wait took, in microseconds.  No fault and no hang is involved. */
+int flux_selftest_bounded_wait(flux_ctx* ctx, int spin_limit_ms, int* waited_us,
+                               flux_stream_t stream);
+
 /* --------------------------------------------------------------------------
  * Layer Router (gist.science summary "Flux Attention", section 2
  * "Methodology": "Layer Router" pools the first and last 100 prompt tokens

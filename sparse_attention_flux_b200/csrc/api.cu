@@ -736,3 +736,13 @@ extern "C" int flux_attn_decode_heads(flux_ctx* c, const uint16_t* q, const uint
   const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_heads: launch");
 }
+
+// ---------------------------------------------------------------------------
+extern "C" int flux_selftest_bounded_wait(flux_ctx* c, int spin_limit_ms, int* waited_us,
+                                          flux_stream_t stream) {
+  if (!c || spin_limit_ms < 1 || spin_limit_ms > 10000)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_selftest_bounded_wait: spin limit in [1, 10000] ms");
+  flux::DevStatus st{c->err, static_cast<long long>(spin_limit_ms) * 1000000LL};
+  const cudaError_t e = flux::launch_selftest_wait(st, waited_us, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_selftest_bounded_wait: launch");
+}

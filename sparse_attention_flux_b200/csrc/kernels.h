@@ -83,6 +83,9 @@ cudaError_t launch_ring_write(const uint16_t* k_src, const uint16_t* v_src, int 
                               uint16_t* v_ring, int sink, int window, int block, int* err,
                               cudaStream_t stream);
 
+// One thread waits on an mbarrier that is never arrived at (bounded wait test).
+cudaError_t launch_selftest_wait(DevStatus st, int* waited_us, cudaStream_t stream);
+
 cudaError_t launch_streaming_mask(int nqb, int nkb, int sink, int window, uint8_t* mask,
                                   cudaStream_t stream);
 cudaError_t launch_block_index(const uint8_t* mask, int nqb, int nkb, int32_t* row_ptr,

@@ -64,6 +64,7 @@ _SIGNATURES = {
                                  _i, _i, _f, _vp], _i),
     "flux_attn_decode_heads": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i, _i,
                                 _i, _f, _vp], _i),
+    "flux_selftest_bounded_wait": ([_vp, _i, _vp, _vp], _i),
     "flux_kv_write": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "flux_attn_decode_sa_compact": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                      _f, _vp], _i),
@@ -163,6 +164,11 @@ class Context:
 
     def set_spin_limit_ms(self, ms: int) -> None:
         _check(lib().flux_ctx_set_spin_limit_ms(self._h, int(ms)))
+
+    def selftest_bounded_wait(self, spin_limit_ms: int, waited_us=None, stream=None) -> None:
+        """Launch a wait that can never complete; the bounded wait must give up."""
+        _check(lib().flux_selftest_bounded_wait(self._h, int(spin_limit_ms), _ptr(waited_us),
+                                                _stream(stream)))
 
     def decode_workspace_bytes(self, B, Hq, Hkv, d, S_max, sink_blocks, window_blocks, block) -> int:
         n = ctypes.c_size_t()
