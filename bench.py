@@ -444,6 +444,26 @@ def run_flux(args, rank, world, dev_index):
     e2e_serial_ms = ranks_max(s0.elapsed_time(s1) / e2e_steps)
     e2e_serial_value = whole_job_rate(wl.flops, world, e2e_serial_ms)
 
+    # router latency: the step's router, and the 36-layer router (hidden 65536 x 2560,
+    # MLP 5120 -> 512 -> 36); CUDA events around 20 back-to-back calls.
+    def time_router(hid, W1, b1, W2, b2, mode):
+        ctx.route(hid, W1, b1, W2, b2, 0.5, mode)
+        a_, b_ = new_ev(), new_ev()
+        a_.record()
+        for _ in range(20):
+            ctx.route(hid, W1, b1, W2, b2, 0.5, mode)
+        b_.record()
+        b_.synchronize()
+        return a_.elapsed_time(b_) / 20 * 1e3
+    router_us = time_router(wl.hidden, wl.W1, wl.b1, wl.W2, wl.b2, wl.mode)
+    h36, W1_36, b1_36, W2_36, b2_36 = synth.router_inputs(65536, HD, H1, 36, synth.seed_for(2),
+                                                          coin_bias=2.0)
+    mode36 = torch.empty(36, dtype=torch.uint8, device=dev)
+    router36_us = time_router(synth.torch_from_bits(h36).to(dev),
+                              *(torch.from_numpy(x).to(dev) for x in (W1_36, b1_36, W2_36, b2_36)),
+                              mode36)
+    del h36
+
     # soft-routing forward blend on the same layer: FA pass + SA pass with a blend epilogue
     score = torch.tensor([0.3], dtype=torch.float32, device=dev)
     soft = lambda: ctx.attn_prefill_soft(wl.q, wl.k, wl.v, wl.o[0], wl.scale, score, 0,
@@ -527,6 +547,9 @@ def run_flux(args, rank, world, dev_index):
                        "frac": round(sa_tflops / peak_t, 4)},
         "fa_prefill": {"TFLOP/s": round(fa_tflops, 1), "ms": round(fa_avg, 4)},
         "soft_prefill": soft_line,
+        "router": {"step_router_us": round(router_us, 2), "router_36_layers_us": round(router36_us, 2),
+                   "per_layer_us_36": round(router36_us / 36, 3),
+                   "context": "pages: 0.20 ms per layer (hardware not stated)"},
         "decode": dec,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,

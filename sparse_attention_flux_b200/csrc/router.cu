@@ -8,9 +8,9 @@
 //   pool_kernel   grid (Hd/256 column groups, 2 sides): each thread sums
 //                 16-byte bf16 vectors of its rows, fixed-order shared-memory
 //                 reduction -> pooled[2 Hd] (fp32).
-//   mlp_kernel    one warp per hidden unit: u = relu(W1 p + b1) with W1 rows
-//                 streamed by 128-bit loads; the last CTA (atomic ticket, no
-//                 spin) computes z = W2 u + b2, r = sigmoid(z) and
+//   mlp_kernel    four warps per hidden unit: u = relu(W1 p + b1) with W1 rows
+//                 streamed by unrolled 128-bit loads; the last CTA (atomic
+//                 ticket, no spin) computes z = W2 u + b2, r = sigmoid(z) and
 //                 layer_mode = (r > thresh).
 #include "common.cuh"
 #include "kernels.h"
@@ -21,6 +21,8 @@ namespace {
 
 constexpr int kPoolThreads = 256;  // 32 column groups of 8 x 8 row groups
 constexpr int kMlpWarps = 8;
+constexpr int kWarpsPerRow = 4;
+constexpr int kRowsPerCta = kMlpWarps / kWarpsPerRow;
 
 __global__ void __launch_bounds__(kPoolThreads)
     pool_kernel(const uint16_t* __restrict__ hidden, int T, int Hd, int n_pool,
@@ -69,26 +71,41 @@ __global__ void __launch_bounds__(kMlpWarps * 32)
                const float* __restrict__ b2, int L, float thresh, float* __restrict__ hidden1,
                int* ticket, uint8_t* __restrict__ layer_mode, float* __restrict__ score) {
   __shared__ int last;
+  __shared__ float part[kMlpWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * kMlpWarps + warp;
+  // kRowsPerCta hidden units per CTA, kWarpsPerRow warps share one unit's dot product.
+  const int j = blockIdx.x * kRowsPerCta + warp / kWarpsPerRow;
+  const int wr = warp % kWarpsPerRow;
+  float acc = 0.f;
   if (j < H1) {
     const float* w = W1 + static_cast<size_t>(j) * in_dim;
-    float acc = 0.f;
     if ((in_dim & 3) == 0) {
-      for (int i = lane * 4; i < in_dim; i += 128) {
-        const float4 wv = __ldg(reinterpret_cast<const float4*>(w + i));
-        const float4 pv = *reinterpret_cast<const float4*>(pooled + i);
+      const int n4 = in_dim >> 2;
+#pragma unroll 4
+      for (int i4 = wr * 32 + lane; i4 < n4; i4 += 32 * kWarpsPerRow) {
+        const float4 wv = __ldg(reinterpret_cast<const float4*>(w) + i4);
+        const float4 pv = *(reinterpret_cast<const float4*>(pooled) + i4);
         acc = fmaf(wv.x, pv.x, acc);
         acc = fmaf(wv.y, pv.y, acc);
         acc = fmaf(wv.z, pv.z, acc);
         acc = fmaf(wv.w, pv.w, acc);
       }
     } else {
-      for (int i = lane; i < in_dim; i += 32) acc = fmaf(__ldg(w + i), pooled[i], acc);
+      for (int i = wr * 32 + lane; i < in_dim; i += 32 * kWarpsPerRow)
+        acc = fmaf(__ldg(w + i), pooled[i], acc);
     }
+  }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) hidden1[j] = fmaxf(acc + b1[j], 0.f);
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) part[warp] = acc;
+  __syncthreads();
+  if (threadIdx.x < kRowsPerCta) {
+    const int jj = blockIdx.x * kRowsPerCta + threadIdx.x;
+    if (jj < H1) {
+      float t = 0.f;
+      for (int q = 0; q < kWarpsPerRow; ++q) t += part[threadIdx.x * kWarpsPerRow + q];
+      hidden1[jj] = fmaxf(t + b1[jj], 0.f);
+    }
   }
   __threadfence();
   __syncthreads();
@@ -123,7 +140,7 @@ cudaError_t launch_route(const RouteLaunch& p, cudaStream_t stream) {
   pool_kernel<<<pgrid, kPoolThreads, 0, stream>>>(p.hidden, p.T, p.Hd, p.n_pool, p.pooled);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int grid = (p.H1 + kMlpWarps - 1) / kMlpWarps;
+  const int grid = (p.H1 + kRowsPerCta - 1) / kRowsPerCta;
   mlp_kernel<<<grid, kMlpWarps * 32, 0, stream>>>(p.pooled, 2 * p.Hd, p.W1, p.b1, p.H1, p.W2,
                                                   p.b2, p.L, p.thresh, p.hidden1, p.ticket,
                                                   p.layer_mode, p.score);
