@@ -2,6 +2,8 @@
 
     python -m sparse_attention_flux_b200.profile_case prefill --mode fa --T 16384 --iters 3
     python -m sparse_attention_flux_b200.profile_case decode --mode sa --B 4 --S 32768
+    python -m sparse_attention_flux_b200.profile_case decode --mode ring --B 16 --S 131072
+    python -m sparse_attention_flux_b200.profile_case append --mode ring --B 16 --S 131072
 
 Inputs are seeded N(0, 1) bf16 drawn on the device; nothing is checked here
 (the test suite does that).  Prints the CUDA-event time per launch.
@@ -19,8 +21,9 @@ from sparse_attention_flux_b200.flux import Context
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["prefill", "decode", "route"])
-    ap.add_argument("--mode", choices=["fa", "sa"], default="fa")
+    ap.add_argument("kernel", choices=["prefill", "decode", "route", "append"])
+    ap.add_argument("--mode", choices=["fa", "sa", "ring"], default="fa",
+                    help="ring: SA decode / append over the compact sink + window cache")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--T", type=int, default=16384)
     ap.add_argument("--S", type=int, default=32768)
@@ -36,6 +39,8 @@ def main() -> None:
     dev = torch.device("cuda", 0)
     ctx = Context(0, 512 << 20)
     mode = torch.tensor([1 if args.mode == "fa" else 0], dtype=torch.uint8, device=dev)
+    if args.kernel == "prefill" and args.mode == "ring":
+        ap.error("--mode ring applies to decode and append")
     scale = 1.0 / math.sqrt(args.d)
     if args.kernel == "prefill":
         B, T = args.B, args.T
@@ -51,16 +56,27 @@ def main() -> None:
         ctx.build_block_index(m, rp, col)
         run = lambda: ctx.attn_prefill(q, k, v, o, scale, layer_mode=mode, row_ptr=rp, col=col,
                                        block=args.block)
-    elif args.kernel == "decode":
+    elif args.kernel in ("decode", "append"):
         B, S = args.B, args.S
+        rows = (args.sink + args.window) * args.block if args.mode == "ring" else S
         q = synth.torch_normal_bf16((B, args.Hq, args.d), 1, dev)
-        kc = synth.torch_normal_bf16((B, S, args.Hkv, args.d), 2, dev)
-        vc = synth.torch_normal_bf16((B, S, args.Hkv, args.d), 3, dev)
+        kc = synth.torch_normal_bf16((B, rows, args.Hkv, args.d), 2, dev)
+        vc = synth.torch_normal_bf16((B, rows, args.Hkv, args.d), 3, dev)
         sl = torch.full((B,), S, dtype=torch.int32, device=dev)
         o = torch.empty_like(q)
-        run = lambda: ctx.attn_decode(q, kc, vc, sl, o, scale, layer_mode=mode,
-                                      sink_blocks=args.sink, window_blocks=args.window,
-                                      block=args.block)
+        if args.kernel == "append":
+            nk = synth.torch_normal_bf16((B, 1, args.Hkv, args.d), 4, dev)
+            nv = synth.torch_normal_bf16((B, 1, args.Hkv, args.d), 5, dev)
+            ring = args.mode == "ring"
+            run = lambda: ctx.kv_write(nk, nv, sl, kc, vc, args.sink if ring else 0,
+                                       args.window if ring else 0, args.block)
+        elif args.mode == "ring":
+            run = lambda: ctx.attn_decode_sa_compact(q, kc, vc, sl, o, scale, args.sink,
+                                                     args.window, args.block)
+        else:
+            run = lambda: ctx.attn_decode(q, kc, vc, sl, o, scale, layer_mode=mode,
+                                          sink_blocks=args.sink, window_blocks=args.window,
+                                          block=args.block)
     else:
         T, Hd, H1, L = args.T, 2560, 512, 36
         hidden = synth.torch_normal_bf16((T, Hd), 1, dev)
