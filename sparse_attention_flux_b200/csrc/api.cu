@@ -375,7 +375,7 @@ int flux_attn_decode(flux_ctx* c, const uint16_t* q, const uint16_t* k_cache,
     return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: tensors must be 16-byte aligned");
   flux::DecodeLaunch p;
   flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
-                    &p.chunk_fa, &p.chunk_sa);
+                    &p.chunk_fa, &p.tiles_sa);
   const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
   const size_t o_bytes = align256(rows * d * sizeof(float));
   const size_t need = o_bytes + align256(rows * 2 * sizeof(float));
@@ -455,7 +455,7 @@ int flux_attn_decode_sa_compact(flux_ctx* c, const uint16_t* q, const uint16_t* 
   const int rows = (sink_blocks + window_blocks) * block;
   flux::DecodeLaunch p;
   flux::decode_plan(B, Hkv, rows, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
-                    &p.chunk_fa, &p.chunk_sa);
+                    &p.chunk_fa, &p.tiles_sa);
   const size_t nrow = static_cast<size_t>(B) * Hq * p.nsplit;
   const size_t o_bytes = align256(nrow * d * sizeof(float));
   if (o_bytes + align256(nrow * 2 * sizeof(float)) > c->workspace_bytes)
@@ -575,7 +575,7 @@ extern "C" int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cac
   if (rc != FLUX_OK) return rc;
   flux::DecodeLaunch p;
   flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, dev->num_sms, &p.nsplit,
-                    &p.chunk_fa, &p.chunk_sa);
+                    &p.chunk_fa, &p.tiles_sa);
   const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
   const size_t ml_bytes = align256(rows * 2 * sizeof(float));
   const size_t o_bytes = align256(rows * d * sizeof(float));
@@ -703,7 +703,7 @@ extern "C" int flux_attn_decode_heads(flux_ctx* c, const uint16_t* q, const uint
     return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: tensors must be 16-byte aligned");
   flux::DecodeLaunch p;
   flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
-                    &p.chunk_fa, &p.chunk_sa);
+                    &p.chunk_fa, &p.tiles_sa);
   const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
   const size_t o_bytes = align256(rows * d * sizeof(float));
   if (o_bytes + align256(rows * 2 * sizeof(float)) > c->workspace_bytes)

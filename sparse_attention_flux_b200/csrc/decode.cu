@@ -53,36 +53,61 @@ struct DSmem {
   static_assert(CO + kComputeWarps * 4 * D * 4 <= BARS, "combine area must fit in the ring");
 };
 
+// A split's 64-token tiles.  FA: a contiguous token range.  SA: the sink
+// segment [0, n_sink) and the window segment [win_start, s) are tiled
+// separately and their tiles numbered consecutively (sink tiles first); split i
+// takes tiles [i * tiles_sa, (i + 1) * tiles_sa), so one split may hold sink
+// tiles followed by window tiles.
 struct Range {
-  int start, end;  // tokens [start, end) of this split
-  int n_active;    // active splits of this (sequence, kv head)
+  bool fa;
+  int start, end;    // FA: tokens [start, end)
+  int v0, v1;        // SA: virtual tiles [v0, v1)
+  int t_sink;        // SA: tiles of the sink segment
+  int n_sink;        // SA: tokens of the sink segment
+  int win_start, s;  // SA: window segment [win_start, s)
+  int ntiles;
+  int n_active;      // active splits of this (sequence, kv head)
+  // Tile k of this split: tokens [*t0, *t1).
+  __device__ __forceinline__ void tile(int k, int* t0, int* t1) const {
+    if (fa) {
+      *t0 = start + k * 64;
+      *t1 = end;
+    } else {
+      const int vt = v0 + k;
+      if (vt < t_sink) {
+        *t0 = vt * 64;
+        *t1 = n_sink;
+      } else {
+        *t0 = win_start + (vt - t_sink) * 64;
+        *t1 = s;
+      }
+    }
+  }
 };
 
 __device__ __forceinline__ Range split_range(const DecodeLaunch& a, bool fa, int s, int i) {
-  Range r{0, 0, 0};
+  Range r{};
+  r.fa = fa;
   if (s <= 0) return r;
   if (fa) {
     r.n_active = (s + a.chunk_fa - 1) / a.chunk_fa;
     r.start = i * a.chunk_fa;
     r.end = min(r.start + a.chunk_fa, s);
+    r.ntiles = r.end > r.start ? (r.end - r.start + kTok - 1) / kTok : 0;
   } else {
     const int blk = a.block;
-    const int n_sink = min(a.sink_blocks * blk, s);
+    r.s = s;
+    r.n_sink = min(a.sink_blocks * blk, s);
     const int nbs = (s + blk - 1) / blk;
-    const int win_start = max(n_sink, max(0, nbs - a.window_blocks) * blk);
-    const int n_win = s - win_start;
-    const int sp_sink = (n_sink + a.chunk_sa - 1) / a.chunk_sa;
-    const int sp_win = (n_win + a.chunk_sa - 1) / a.chunk_sa;
-    r.n_active = sp_sink + sp_win;
-    if (i < sp_sink) {
-      r.start = i * a.chunk_sa;
-      r.end = min(r.start + a.chunk_sa, n_sink);
-    } else if (i < r.n_active) {
-      r.start = win_start + (i - sp_sink) * a.chunk_sa;
-      r.end = min(r.start + a.chunk_sa, s);
-    }
+    r.win_start = max(r.n_sink, max(0, nbs - a.window_blocks) * blk);
+    r.t_sink = (r.n_sink + kTok - 1) / kTok;
+    const int total = r.t_sink + (s - r.win_start + kTok - 1) / kTok;
+    r.n_active = (total + a.tiles_sa - 1) / a.tiles_sa;
+    r.v0 = i * a.tiles_sa;
+    r.v1 = min(r.v0 + a.tiles_sa, total);
+    r.ntiles = r.v1 > r.v0 ? r.v1 - r.v0 : 0;
   }
-  if (i >= r.n_active) r.start = r.end = 0;
+  if (i >= r.n_active) r.ntiles = 0;
   return r;
 }
 
@@ -119,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     s = 0;
   }
   const Range rg = split_range(a, fa, s, i);
-  const int ntiles = (rg.end - rg.start + kTok - 1) / kTok;
+  const int ntiles = rg.ntiles;
   const size_t grp = static_cast<size_t>(b) * a.Hq + g * G;  // first query head of the group
   if (ntiles == 0) {
     // Splits past the active range exit at once (SA layers use only a few);
@@ -164,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint8_t* kb = smem + st * L::STAGE;
         uint8_t* vb = kb + L::KT;
         mbar_arrive_expect_tx(&full[st], 2 * L::KT);
-        int row = rg.start + k * kTok;
+        int row, t_end;
+        rg.tile(k, &row, &t_end);
         if (a.compact && row >= a.sink_blocks * a.block) {
           // Ring slot of the token's block (a 64-token tile never straddles blocks).
           const int j = row / a.block;
@@ -223,7 +249,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       // ---- online softmax on the fragment: row gq, tokens 8n + 2tq + e
-      const int tok0 = rg.start + k * kTok + wtok + 2 * tq;
+      int t_begin, t_end;
+      rg.tile(k, &t_begin, &t_end);
+      const int tok0 = t_begin + wtok + 2 * tq;
       float x[4];
 #pragma unroll
       for (int n = 0; n < 2; ++n)
@@ -231,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int e = 0; e < 2; ++e)
         {
           const int u = tok0 + 8 * n + e;
-          const bool keep = gq < G && u < rg.end &&
+          const bool keep = gq < G && u < t_end &&
                             (!row_sa || u / a.block < a.sink_blocks ||
                              u / a.block >= nbs - a.window_blocks);
           x[n * 2 + e] = keep ? sc[n][e] : -INFINITY;
@@ -370,35 +398,33 @@ cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeL
 }  // namespace
 
 void decode_plan(int B, int Hkv, int S_max, int sink_blocks, int window_blocks, int block,
-                 int num_sms, int* nsplit, int* chunk_fa, int* chunk_sa) {
-  // FA: chunks of about 2048 tokens (1 MiB of K+V per CTA at d=128), but at
-  // least ~4 CTAs per SM in total; never below one 64-token tile.
+                 int num_sms, int* nsplit, int* chunk_fa, int* tiles_sa) {
   const long long groups = static_cast<long long>(B) * Hkv;
+  const long long slots = 2LL * num_sms;   // two CTAs per SM
+  // FA: chunks of about 2048 tokens (1 MiB of K+V per CTA at d=128), but at
+  // least ~2 waves of CTAs in total; never below one 64-token tile.
   int ns = (S_max + 2047) / 2048;
-  const int want = static_cast<int>((4LL * num_sms + groups - 1) / groups);
+  const int want = static_cast<int>((2 * slots + groups - 1) / groups);
   if (ns < want) ns = want;
   const int max_ns = (S_max + kTok - 1) / kTok;
   if (ns > max_ns) ns = max_ns;
   if (ns < 1) ns = 1;
-  int cfa = (S_max + ns - 1) / ns;
-  cfa = ((cfa + kTok - 1) / kTok) * kTok;
-  // SA: the sink + window tokens, in chunks of at least one tile, spread over
-  // about 8 splits.
-  const long long sa_tokens = static_cast<long long>(sink_blocks + window_blocks) * block;
-  long long csa = (sa_tokens + 7) / 8;
-  csa = ((csa + kTok - 1) / kTok) * kTok;
-  if (csa < kTok) csa = kTok;
-  if (csa < cfa / 64) csa = ((cfa / 64 + kTok - 1) / kTok) * kTok;
-  // The split count must cover both modes for any seqlen <= S_max.
-  const long long need_sa = (static_cast<long long>(sink_blocks) * block + csa - 1) / csa +
-                            (static_cast<long long>(window_blocks) * block + csa - 1) / csa;
+  // SA: the sink and window tiles of a sequence, spread so that an SA layer's
+  // active CTAs fill about one wave.
+  const long long sa_tiles = (static_cast<long long>(sink_blocks) * block + kTok - 1) / kTok +
+                             (static_cast<long long>(window_blocks) * block + kTok - 1) / kTok;
+  long long sa_splits = (slots + groups - 1) / groups;
+  if (sa_splits < 1) sa_splits = 1;
+  if (sa_splits > sa_tiles) sa_splits = sa_tiles;
+  const long long tsa = (sa_tiles + sa_splits - 1) / sa_splits;
+  const long long need_sa = (sa_tiles + tsa - 1) / tsa;
   ns = static_cast<int>(std::max<long long>(ns, need_sa));
-  cfa = (S_max + ns - 1) / ns;
+  int cfa = (S_max + ns - 1) / ns;
   cfa = ((cfa + kTok - 1) / kTok) * kTok;
   if (cfa < kTok) cfa = kTok;
   *nsplit = ns;
   *chunk_fa = cfa;
-  *chunk_sa = static_cast<int>(csa);
+  *tiles_sa = static_cast<int>(tsa);
 }
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int nsplit) {

@@ -44,7 +44,7 @@ struct DecodeLaunch {
   int layer;
   int sink_blocks, window_blocks, block;
   float scale;
-  int nsplit, chunk_fa, chunk_sa;
+  int nsplit, chunk_fa, tiles_sa;   // FA tokens per split; SA 64-token tiles per split
   int compact;      // SA over the compact ring cache (sink + window blocks), S_max = ring rows
   const uint8_t* head_mode;  // per-query-head routing [Hq] (overrides layer_mode), or null
   float* part_o;    // [B, Hq, nsplit, d]
@@ -54,7 +54,7 @@ struct DecodeLaunch {
 };
 // Split plan for a shape (host only): number of splits and chunk lengths.
 void decode_plan(int B, int Hkv, int S_max, int sink_blocks, int window_blocks, int block,
-                 int num_sms, int* nsplit, int* chunk_fa, int* chunk_sa);
+                 int num_sms, int* nsplit, int* chunk_fa, int* tiles_sa);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int nsplit);
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeLaunch& p,
                           cudaStream_t stream);
