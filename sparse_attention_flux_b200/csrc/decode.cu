@@ -202,13 +202,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         issued = k + 1;
       }
-      if (!ok) {
-        // Let the copies still in flight land before the CTA's smem goes away.
-        DevStatus drain = a.st;
-        drain.spin_ns = 100000000;
-        for (int k = max(0, issued - kStages); k < issued; ++k)
-          mbar_wait(&full[k % kStages], (k / kStages) & 1, drain);
-      }
+      // Every copy issued lands before the ring is reused for the merge, also
+      // when the compute warps gave up early.
+      for (int k = max(0, issued - kStages); k < issued; ++k)
+        mbar_drain(&full[k % kStages], (k / kStages) & 1);
     }
   } else if (ntiles > 0) {
     // ------------------------------------------------------------ compute warps

@@ -3,11 +3,16 @@
 // Flux Attention routes each layer to Full Attention (exact causal softmax
 // attention) or to block-sparse Sparse Attention (arXiv abstract; model card
 // "Flux Attention: Qwen3-4B", "Sample Usage").  One kernel serves both: a
-// CTA owns 256 query rows -- two 128-row tiles Q0, Q1 -- of one (batch, query
-// head) and walks a list of 128-column key tiles: every tile up to the
-// diagonal for FA, the tiles named by the compressed block-index list for SA
-// (built once per CTA into shared memory), so skipped blocks are never loaded.
-// Each K/V tile is loaded once and used by both query tiles.
+// CTA owns two 128-row query tiles Q0, Q1 that read the same keys and walks a
+// list of 128-column key tiles: every tile up to the diagonal for FA, the
+// tiles named by the compressed block-index list for SA (built once per CTA
+// into shared memory), so skipped blocks are never loaded.  Each K/V tile is
+// loaded once and used by both query tiles.  The two tiles are either
+//   a head pair (GQA with an even group size): the same 128 rows of two query
+//     heads that share a KV head.  Both tiles need exactly the same key tiles,
+//     so no MMA or softmax is spent on a tile that only one of them sees; or
+//   a row pair (odd group size, or per-head routing): rows [256u, 256u + 256)
+//     of one query head, walking the union of the two tiles' lists.
 //
 // Per CTA (384 threads, warp-specialised):
 //   warp 0      TMA producer (Q0, Q1 once; K/V tiles into a 2-stage ring) and,
@@ -40,7 +45,8 @@ constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold, log2 units
 
 struct PrefillArgs {
   int B, T, Hq, Hkv, G;
-  int npair;         // 256-row query pairs along T
+  int head_pair;     // 1: a CTA = one 128-row tile of two heads; 0: 256 rows of one head
+  int nunit;         // CTA units along T: 128-row tiles (head pair) or 256-row pairs
   int nkt;           // 128-column key tiles along T
   int block;         // mask block: 64 or a multiple of 128
   int nqb;           // rows of the CSR
@@ -78,18 +84,19 @@ struct Smem {
 
 // SA: the CTA's key tiles and, per tile, which (64-row query sub-block,
 // 64-column key sub-block) pairs the block mask keeps: bit (qs * 2 + ks).
-// One warp: OR every kept block of the (up to four) CSR rows the CTA's query
-// rows fall in into a per-tile map, then compact it in ascending tile order.
-// Returns the list length.  Tiles past the last query row's diagonal are
-// dropped (causal), CSR entries out of range raise DEV_ERR_CSR and are skipped.
-__device__ int build_tile_list(const PrefillArgs& a, int pair, uint32_t* map, uint32_t* list) {
+// One warp: OR every kept block of the CSR rows that the CTA's nsub 64-row
+// sub-blocks (from row0) fall in into a per-tile map, then compact it in
+// ascending tile order.  Returns the list length.  Tiles past the last tile
+// index `last` (the diagonal) are dropped (causal); CSR entries out of range
+// raise DEV_ERR_CSR and are skipped.
+__device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int last, uint32_t* map,
+                               uint32_t* list) {
   const int lane = threadIdx.x & 31;
-  const int last = min(2 * pair + 1, a.nkt - 1);
   for (int J = lane; J <= last; J += 32) map[J] = 0;
   __syncwarp();
   const int nnz = a.row_ptr[a.nqb];
-  for (int qs = 0; qs < 4; ++qs) {
-    const int row = pair * 256 + qs * 64;
+  for (int qs = 0; qs < nsub; ++qs) {
+    const int row = row0 + qs * 64;
     if (row >= a.T) break;
     const int qb = row / a.block;
     if (qb >= a.nqb) {
@@ -148,15 +155,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* nlist = reinterpret_cast<int*>(smem + L::NLIST);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Longest-first order: the last query pairs carry the most causal work.
-  const int per_pair = a.Hq * a.B;
-  const int pair = a.npair - 1 - static_cast<int>(blockIdx.x) / per_pair;
-  const int rem = static_cast<int>(blockIdx.x) % per_pair;
-  const int b = rem / a.Hq, h = rem % a.Hq, g = h / a.G;
+  // Longest-first order: the last query rows carry the most causal work.
+  // Tile i (0, 1) holds rows [row0 + i * row_step, +128) of query head
+  // head0 + i * head_step.
+  const int hpu = a.head_pair ? a.Hq / 2 : a.Hq;   // head units per batch
+  const int per_unit = hpu * a.B;
+  const int unit = a.nunit - 1 - static_cast<int>(blockIdx.x) / per_unit;
+  const int rem = static_cast<int>(blockIdx.x) % per_unit;
+  const int b = rem / hpu, hu = rem % hpu;
+  const int row0 = unit * (a.head_pair ? kBM : 2 * kBM);          // first row of the unit
+  const int nrow = a.head_pair ? kBM : 2 * kBM;                    // rows of the unit
+  const int head0 = a.head_pair ? 2 * hu : hu, head_step = a.head_pair ? 1 : 0;
+  const int row_step = a.head_pair ? 0 : kBM;
+  const int g = head0 / a.G;
   const bool fa = a.force_mode >= 0 ? a.force_mode == 1
-                 : a.head_mode     ? a.head_mode[h] != 0
+                 : a.head_mode     ? a.head_mode[hu] != 0
                                    : (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
-  const int q0 = pair * 256;
+  const int last_tile = min((row0 + nrow - 1) / kBN, a.nkt - 1);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_Q], 1);
@@ -170,9 +185,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[B_OD], 1);
     mbar_init(&bars[B_DRAIN], 1);
     fence_barrier_init();
+    fence_proxy_async_smem();
+    // Q does not depend on the key-tile list: start it now, so that its
+    // latency overlaps the list build (two dependent global reads).
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    mbar_arrive_expect_tx(&bars[B_Q], 2 * CH * kChunkBytes);
+    for (int i = 0; i < 2; ++i)
+      for (int c = 0; c < CH; ++c)
+        tma_load_4d(&tm_q, &bars[B_Q], sQ + (i * CH + c) * kChunkBytes, c * 64,
+                    head0 + i * head_step, row0 + i * row_step, b);
   }
   if (warp == 0) {
-    const int n = fa ? min(2 * pair + 1, a.nkt - 1) + 1 : build_tile_list(a, pair, map, list);
+    const int n = fa ? last_tile + 1 : build_tile_list(a, row0, nrow / 64, last_tile, map, list);
     if (lane == 0) *nlist = n;
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -193,15 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars[B_Q], 2 * CH * kChunkBytes);
-      for (int i = 0; i < 2; ++i)
-        for (int c = 0; c < CH; ++c)
-          tma_load_4d(&tm_q, &bars[B_Q], sQ + (i * CH + c) * kChunkBytes, c * 64, h,
-                      q0 + i * kBM, b);
+    if (lane == 0) {
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
@@ -219,15 +237,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                       J * kBN, b);
         issued = j + 1;
       }
-      if (!ok) {
-        // Let the copies already issued land before the CTA's smem goes away.
-        DevStatus drain = a.st;
-        drain.spin_ns = 100000000;  // 100 ms
-        mbar_wait(&bars[B_Q], 0, drain);
-        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
-          mbar_wait(&bars[B_KF + (j & 1)], (j >> 1) & 1, drain);
-          mbar_wait(&bars[B_VF + (j & 1)], (j >> 1) & 1, drain);
-        }
+      // Every copy issued lands before the CTA's smem goes away, also when a
+      // consumer gave up early (loads before the last two were consumed).
+      mbar_drain(&bars[B_Q], 0);
+      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
+        mbar_drain(&bars[B_KF + (j & 1)], (j >> 1) & 1);
+        mbar_drain(&bars[B_VF + (j & 1)], (j >> 1) & 1);
       }
     }
   } else if (warp == 1) {
@@ -286,17 +301,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) umma_commit(&bars[B_OD]);
       // Every MMA issued by this thread is complete before TMEM is released.
       umma_commit(&bars[B_DRAIN]);
-      DevStatus drain = a.st;
-      drain.spin_ns = 100000000;
-      mbar_wait(&bars[B_DRAIN], 0, drain);
+      mbar_drain(&bars[B_DRAIN], 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax
     const int i = (warp - 4) >> 2;           // query tile 0 or 1
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int r = quarter * 32 + lane;       // row within the tile
-    const int t_row = q0 + i * kBM + r;
-    const int qs = (i * kBM + r) >> 6;       // 64-row sub-block within the pair
+    const int t_row = row0 + i * row_step + r;
+    const int h = head0 + i * head_step;
+    const int qs = (t_row - row0) >> 6;      // 64-row sub-block within the unit
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + i * 128;
     const uint32_t tO = tmem + lane_off + 256 + i * 128;
@@ -455,7 +469,9 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   a.Hq = p.Hq;
   a.Hkv = p.Hkv;
   a.G = p.Hq / p.Hkv;
-  a.npair = (p.T + 255) / 256;
+  // Head pairs need both heads of a pair in one KV group and on one path.
+  a.head_pair = (a.G % 2 == 0 && p.head_mode == nullptr) ? 1 : 0;
+  a.nunit = a.head_pair ? (p.T + kBM - 1) / kBM : (p.T + 2 * kBM - 1) / (2 * kBM);
   a.nkt = (p.T + kBN - 1) / kBN;
   a.block = p.block;
   a.nqb = p.nqb;
@@ -471,7 +487,7 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   a.head_mode = p.head_mode;
   a.blend_score = p.blend_score;
   a.st = p.st;
-  const dim3 grid(static_cast<unsigned>(a.npair) * p.Hq * p.B);
+  const dim3 grid(static_cast<unsigned>(a.nunit) * (a.head_pair ? p.Hq / 2 : p.Hq) * p.B);
   if (p.d == 64) {
     const int smem = Smem<64>::ALLOC;
     cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

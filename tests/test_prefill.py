@@ -70,6 +70,8 @@ CASES = [  # B, T, Hq, Hkv, d, block, sink, W
     (1, 700, 2, 2, 64, 64, 1, 3),
     (1, 1000, 4, 4, 128, 256, 1, 2),
     (1, 1500, 8, 2, 128, 128, 0, 4),
+    (1, 777, 6, 2, 128, 128, 1, 3),     # odd group size (3): row-pair CTAs
+    (2, 384, 12, 2, 64, 64, 2, 2),      # group size 6: head-pair CTAs across three pairs
 ]
 
 
