@@ -15,7 +15,12 @@ pair per head) / step time.  The decode half of the metric (KV GB/s) is timed
 in the same run on the 36-layer Qwen3-4B-shaped decode workload (batch 16, KV
 131072 + step, 18 FA / 18 SA layers, 64 steps; every layer appends the new token's
 K/V -- the full cache of an FA layer, the compact sink + window ring of an SA layer -- and
-decodes) and reported under "decode".
+decodes) and reported under "decode", with one SA ring layer timed alone with and
+without an L2 flush.  On one GPU the line also carries, each timed in a few seconds,
+"prefill_36_layers" (the routed 36-layer prefill at T 65536: router, mask, CSR, 36
+layers reading their bits on the device) and "llama_3_1_8b" (32-layer shapes:
+prefill FA and SA layers at T 131072 for windows of 8/16/32 blocks; 32-layer decode
+at B 4, S 131072 for 0-100 % SA layers); --no-extended skips them.
 
 Every input is seeded and synthetic; every timed input (640 MB for prefill,
 17 GB of KV for decode) is larger than the 126 MB L2, so no flush is needed.
@@ -362,6 +367,36 @@ class DecodeWorkload:
         out["sa_fraction"] = 0.5
         return out
 
+    def sa_layer(self, reps):
+        """One SA layer's decode over its compact ring (B 16, the last step's length), timed
+        launch by launch: back to back (ring partly L2-resident: 143 MB of K+V against a
+        126 MB L2) and with a 256 MB write between launches (cold L2)."""
+        import torch
+        layer = min(self.rings)
+        kr, vr = self.rings[layer]
+        sl = self.seqlens[-1]
+        s = DEC_S + self.steps
+        byts = DEC_B * sa_decode_tokens(s, BLOCK, SINK, WIN) * HKV * D * 2 * 2
+        fn = lambda: self.ctx.attn_decode_sa_compact(self.q, kr, vr, sl, self.o, self.scale,
+                                                     SINK, WIN, BLOCK)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=self.dev)
+        out = {}
+        for name, flushed in (("unflushed", False), ("flushed", True)):
+            evs = _events(torch, reps)
+            fn()
+            for i, (a, b) in enumerate(evs):
+                if flushed:
+                    flush.fill_(i & 0xFF)
+                a.record()
+                fn()
+                b.record()
+            torch.cuda.synchronize()
+            us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+            out[name] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1)}
+        out["kv_bytes"] = byts
+        del flush
+        return out
+
     def capture(self):
         """One 36-layer decode step (72 launches) captured as a CUDA graph; per step the
         device seqlens are updated and the graph replayed."""
@@ -399,6 +434,182 @@ class DecodeWorkload:
                 kr, vr = self.rings[layer]
                 c.kv_write(self.new_k, self.new_v, sl, kr, vr, SINK, WIN, BLOCK)
                 c.attn_decode_sa_compact(self.q, kr, vr, sl, self.o, self.scale, SINK, WIN, BLOCK)
+
+
+def _events(torch, n):
+    return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(n)]
+
+
+def prefill_36_layers(ctx, dev, seed, reps=2):
+    """36-layer routed prefill, Qwen3-4B shapes at T 65536 (B 1, Hq 32, Hkv 8, d 128):
+    router on hidden 65536 x 2560 (MLP 5120 -> 512 -> 36, b2 = +-2 from a seeded coin:
+    about half the layers SA) -> mask -> CSR -> 36 flux_attn_prefill calls, each reading
+    its layer's bit on the device.  Q/K/V are aliased across layers (805 MB, far above
+    L2); the values do not change the work.  One warm-up pass, then `reps` timed passes."""
+    import torch
+    from sparse_attention_flux_b200 import synth
+    T2, L = 65536, 36
+    q = synth.torch_normal_bf16((1, T2, HQ, D), seed + 1, dev)
+    k = synth.torch_normal_bf16((1, T2, HKV, D), seed + 2, dev)
+    v = synth.torch_normal_bf16((1, T2, HKV, D), seed + 3, dev)
+    o = torch.empty_like(q)
+    h, W1, b1, W2, b2 = synth.router_inputs(T2, HD, H1, L, seed + 4, coin_bias=2.0)
+    hidden = synth.torch_from_bits(h).to(dev)
+    W1, b1, W2, b2 = (torch.from_numpy(x).to(dev) for x in (W1, b1, W2, b2))
+    del h
+    mode = torch.empty(L, dtype=torch.uint8, device=dev)
+    nb = T2 // BLOCK
+    mask = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
+    row_ptr = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(nb * nb, dtype=torch.int32, device=dev)
+    scale = 1.0 / math.sqrt(D)
+
+    def one(evs=None):
+        if evs is not None:
+            evs[0][0].record()
+        ctx.route(hidden, W1, b1, W2, b2, 0.5, mode)
+        ctx.build_streaming_mask(nb, nb, SINK, WIN, mask)
+        ctx.build_block_index(mask, row_ptr, col)
+        if evs is not None:
+            evs[0][1].record()
+        for layer in range(L):
+            if evs is not None:
+                evs[1 + layer][0].record()
+            ctx.attn_prefill(q, k, v, o, scale, layer_mode=mode, layer=layer, row_ptr=row_ptr,
+                             col=col, block=BLOCK)
+            if evs is not None:
+                evs[1 + layer][1].record()
+
+    one()
+    ctx.check()
+    runs = [_events(torch, 1 + L) for _ in range(reps)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for evs in runs:
+        one(evs)
+    b.record()
+    b.synchronize()
+    ctx.check()
+    step_ms = a.elapsed_time(b) / reps
+    mode_h = mode.cpu().numpy()
+    fa_l = [l for l in range(L) if mode_h[l]]
+    sa_l = [l for l in range(L) if not mode_h[l]]
+    per = [[evs[1 + l][0].elapsed_time(evs[1 + l][1]) for l in range(L)] for evs in runs]
+    fa_ms = statistics.mean(p[l] for p in per for l in fa_l) if fa_l else 0.0
+    sa_ms = statistics.mean(p[l] for p in per for l in sa_l) if sa_l else 0.0
+    head_ms = statistics.mean(evs[0][0].elapsed_time(evs[0][1]) for evs in runs)
+    f_fa = 4.0 * D * causal_pairs_fa(T2) * HQ
+    f_sa = 4.0 * D * pairs_sa(T2, BLOCK, SINK, WIN) * HQ
+    flops = len(fa_l) * f_fa + len(sa_l) * f_sa
+    out = {
+        "workload": "qwen3-4b-36L-routed-prefill: B 1, T 65536, Hq 32, Hkv 8, d 128; router "
+                    "65536x2560 -> MLP 5120-512-36 (b2 = +-2, seeded coin); SA block 128, "
+                    "sink 1, window 16; Q/K/V aliased across layers",
+        "fa_layers": len(fa_l), "sa_layers": len(sa_l),
+        "ms_per_step": round(step_ms, 3),
+        "TFLOP/s": round(flops / (step_ms * 1e-3) / 1e12, 1),
+        "fa_layer": {"ms": round(fa_ms, 3),
+                     "TFLOP/s": round(f_fa / (fa_ms * 1e-3) / 1e12, 1) if fa_ms else None},
+        "sa_layer": {"ms": round(sa_ms, 3),
+                     "TFLOP/s": round(f_sa / (sa_ms * 1e-3) / 1e12, 1) if sa_ms else None},
+        "router_mask_csr_us": round(head_ms * 1e3, 1),
+        "timed_passes": reps,
+    }
+    del q, k, v, o, hidden
+    torch.cuda.empty_cache()
+    return out
+
+
+def llama_sweep(ctx, dev, seed):
+    """Llama-3.1-8B shapes (32 layers, Hq 32, Hkv 8, d 128), no router (fixed modes).
+
+    prefill, B 1, T 131072: one FA layer and one SA layer per window W in {8, 16, 32}
+    blocks of 128 (sink 1), each timed over 2 launches after a warm-up; the 32-layer step
+    at each SA fraction is the sum of its layers' measured times (layers are sequential,
+    independent launches whose inputs exceed L2).
+    decode, B 4, S 131072: the whole 32-layer step measured at SA fractions 0/25/50/75/100 %
+    (W 16; seeded layer choice) and at 50 % for W 8 and 32; every layer has its own full
+    cache (2.15 GB; 69 GB in all), so no layer's window is left in L2 by another's."""
+    import torch
+    from sparse_attention_flux_b200 import synth
+    L, T3, B4, S4 = 32, 131072, 4, 131072
+    scale = 1.0 / math.sqrt(D)
+    out = {"workload": "llama-3.1-8b: 32 layers, Hq 32, Hkv 8, d 128; prefill B 1 T 131072; "
+                       "decode B 4 S 131072; sink 1, W in {8, 16, 32} blocks of 128"}
+    # ---- prefill
+    q = synth.torch_normal_bf16((1, T3, HQ, D), seed + 1, dev)
+    k = synth.torch_normal_bf16((1, T3, HKV, D), seed + 2, dev)
+    v = synth.torch_normal_bf16((1, T3, HKV, D), seed + 3, dev)
+    o = torch.empty_like(q)
+    nb = T3 // BLOCK
+    mask = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
+    row_ptr = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(nb * nb, dtype=torch.int32, device=dev)
+    fa_mode = torch.ones(1, dtype=torch.uint8, device=dev)
+    sa_mode = torch.zeros(1, dtype=torch.uint8, device=dev)
+
+    def timed(fn, n=2):
+        fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / n
+
+    ctx.build_streaming_mask(nb, nb, SINK, 16, mask)
+    ctx.build_block_index(mask, row_ptr, col)
+    fa_ms = timed(lambda: ctx.attn_prefill(q, k, v, o, scale, layer_mode=fa_mode, row_ptr=row_ptr,
+                                           col=col, block=BLOCK))
+    f_fa = 4.0 * D * causal_pairs_fa(T3) * HQ
+    pre = {"fa_layer": {"ms": round(fa_ms, 3), "TFLOP/s": round(f_fa / (fa_ms * 1e-3) / 1e12, 1)}}
+    sa_ms_w = {}
+    for W in (8, 16, 32):
+        ctx.build_streaming_mask(nb, nb, SINK, W, mask)
+        ctx.build_block_index(mask, row_ptr, col)
+        sa_ms_w[W] = timed(lambda: ctx.attn_prefill(q, k, v, o, scale, layer_mode=sa_mode,
+                                                    row_ptr=row_ptr, col=col, block=BLOCK))
+        f_sa = 4.0 * D * pairs_sa(T3, BLOCK, SINK, W) * HQ
+        pre[f"sa_layer_W{W}"] = {"ms": round(sa_ms_w[W], 3),
+                                 "TFLOP/s": round(f_sa / (sa_ms_w[W] * 1e-3) / 1e12, 1)}
+    ctx.check()
+    pre["step_ms_by_sa_fraction_W16"] = {
+        f"{pct}%": round((L - L * pct // 100) * fa_ms + (L * pct // 100) * sa_ms_w[16], 1)
+        for pct in (0, 25, 50, 75, 100)}
+    pre["how"] = "per-layer launches timed; 32-layer step = sum of its layers' times"
+    out["prefill"] = pre
+    del q, k, v, o
+    torch.cuda.empty_cache()
+    # ---- decode
+    shape = (B4, S4, HKV, D)
+    caches = [(synth.torch_normal_bf16(shape, seed + 10 * i + 11, dev),
+               synth.torch_normal_bf16(shape, seed + 10 * i + 12, dev)) for i in range(L)]
+    qd = synth.torch_normal_bf16((B4, HQ, D), seed + 30, dev)
+    od = torch.empty_like(qd)
+    sl = torch.full((B4,), S4, dtype=torch.int32, device=dev)
+    kv_row = HKV * D * 2 * 2
+
+    def dec_step(mode_t, W):
+        for layer in range(L):
+            kc, vc = caches[layer]
+            ctx.attn_decode(qd, kc, vc, sl, od, scale, layer_mode=mode_t, layer=layer,
+                            sink_blocks=SINK, window_blocks=W, block=BLOCK)
+
+    dec = {}
+    for pct, W in [(0, 16), (25, 16), (50, 16), (75, 16), (100, 16), (50, 8), (50, 32)]:
+        n_sa = L * pct // 100
+        mode_t = torch.from_numpy(synth.layer_mode_choice(L, L - n_sa, seed + pct)).to(dev)
+        ms = timed(lambda: dec_step(mode_t, W), n=5)
+        byts = B4 * ((L - n_sa) * S4 + n_sa * sa_decode_tokens(S4, BLOCK, SINK, W)) * kv_row
+        dec[f"sa{pct}%_W{W}"] = {"ms_per_step": round(ms, 3),
+                                 "GB/s": round(byts / (ms * 1e-3) / 1e9, 1)}
+    ctx.check()
+    out["decode"] = dec
+    del caches
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_flux(args, rank, world, dev_index):
@@ -557,9 +768,16 @@ def run_flux(args, rank, world, dev_index):
                     "traffic": None, "kernel": "decode_kernel<128,4> (FA layer, incl. its append)"}
         dec["roofline"] = roof_dec
         dec["routing_granularity"] = dw.granularity(8)
+        dec["sa_layer"] = dw.sa_layer(10)
         ctx.check()
         del dw.graph
         del dw
+    torch.cuda.empty_cache()
+    extended = {}
+    if not args.no_extended and world == 1:
+        from sparse_attention_flux_b200 import synth as _s
+        extended["prefill_36_layers"] = prefill_36_layers(ctx, dev, _s.seed_for(2) + 1000 * rank)
+        extended["llama_3_1_8b"] = llama_sweep(ctx, dev, _s.seed_for(4) + 1000 * rank)
     ctx.close()
 
     line = {
@@ -584,6 +802,7 @@ def run_flux(args, rank, world, dev_index):
                    "per_layer_us_36": round(router36_us / 36, 3),
                    "context": "pages: 0.20 ms per layer (hardware not stated)"},
         "decode": dec,
+        **extended,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                 "how": "pinned host -> device copy of Q/K/V/hidden, router + index + FA + SA "
@@ -599,9 +818,13 @@ def run_flux(args, rank, world, dev_index):
     return line
 
 
-def cpu_baseline(seconds_budget=15.0):
-    """The oracle, as it stands, on a bounded sample of the same prefill workload."""
+def cpu_baseline(seconds_budget=15.0, threads=None):
+    """The oracle, as it stands, on a bounded sample of the same prefill workload
+    (all host cores, or `threads` of them)."""
     import oracle
+    if threads is not None:
+        all_threads = oracle.num_threads()
+        oracle.set_num_threads(threads)
     from sparse_attention_flux_b200 import synth
     seed = synth.seed_for(1)
     q, k, v = synth.attention_inputs(1, T, HQ, HKV, D, seed)
@@ -630,7 +853,10 @@ def cpu_baseline(seconds_budget=15.0):
             n_rows += 64
         t_used += time.perf_counter() - t0
     tflops = 4.0 * D * done_pairs / t_used / 1e12
-    return {"value": tflops, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+    cores = oracle.num_threads()
+    if threads is not None:
+        oracle.set_num_threads(all_threads)
+    return {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{n_rows} uniformly sampled query rows (half FA, half SA) of the T=32768 "
                       f"layer, {t_used:.1f} s; FLOPs counted like the GPU's (4 d per visible pair)"}
 
@@ -643,6 +869,8 @@ def main():
     ap.add_argument("--impl", choices=["flux", "reference"], default="flux")
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extended", action="store_true",
+                    help="skip the 36-layer T 65536 prefill and the Llama-3.1-8B sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
@@ -682,6 +910,9 @@ def main():
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+            one = cpu_baseline(4.0, threads=1)
+            line["cpu_baseline"]["single_thread"] = {"value": one["value"], "cores": 1,
+                                                     "sample": one["sample"]}
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

@@ -64,8 +64,11 @@ struct PrefillArgs {
   DevStatus st;
 };
 
-enum { B_Q = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_SF = 7, B_PF = 9, B_OD = 11, B_DRAIN = 12,
-       B_COUNT = 13 };
+// K and V slots are released separately: K(j) once S1(j) has read it, V(j)
+// once PV1(j) has, so the load of K(j+2) starts about a tile-step earlier
+// than it could if both waited for PV1(j).
+enum { B_Q = 0, B_KF = 1, B_VF = 3, B_KE = 5, B_VE = 7, B_SF = 9, B_PF = 11, B_OD = 13,
+       B_DRAIN = 14, B_COUNT = 15 };
 
 template <int D>
 struct Smem {
@@ -179,6 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[B_KF + s], 1);
       mbar_init(&bars[B_VF + s], 1);
       mbar_init(&bars[B_KE + s], 1);
+      mbar_init(&bars[B_VE + s], 1);
       mbar_init(&bars[B_SF + s], 1);
       mbar_init(&bars[B_PF + s], 128);
     }
@@ -231,6 +235,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < CH; ++c)
           tma_load_4d(&tm_k, &bars[B_KF + s], sK + (s * CH + c) * kChunkBytes, c * 64, g,
                       J * kBN, b);
+        if (j >= 2 && !mbar_wait(&bars[B_VE + s], ((j >> 1) - 1) & 1, a.st)) {
+          // K(j) is in flight; V(j) is not: drain only what was issued.
+          mbar_drain(&bars[B_KF + s], (j >> 1) & 1);
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&bars[B_VF + s], CH * kChunkBytes);
         for (int c = 0; c < CH; ++c)
           tma_load_4d(&tm_v, &bars[B_VF + s], sV + (s * CH + c) * kChunkBytes, c * 64, g,
@@ -275,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&bars[B_SF + 0]);
         issue_s(1, 0);
         umma_commit(&bars[B_SF + 1]);
+        umma_commit(&bars[B_KE + 0]);
       }
       for (int j = 0; ok && j < n; ++j) {
         const int s = j & 1, sn = (j + 1) & 1;
@@ -292,10 +303,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bars[B_PF + 1], j & 1, a.st)) { ok = false; break; }
         tc_fence_after();
         issue_pv(1, s, j > 0);
-        umma_commit(&bars[B_KE + s]);
+        umma_commit(&bars[B_VE + s]);
         if (more) {
           issue_s(1, sn);
           umma_commit(&bars[B_SF + 1]);
+          umma_commit(&bars[B_KE + sn]);
         }
       }
       if (ok) umma_commit(&bars[B_OD]);
