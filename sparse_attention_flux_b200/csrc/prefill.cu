@@ -91,26 +91,38 @@ struct Smem {
 // sub-blocks (from row0) fall in into a per-tile map, then compact it in
 // ascending tile order.  Returns the list length.  Tiles past the last tile
 // index `last` (the diagonal) are dropped (causal); CSR entries out of range
-// raise DEV_ERR_CSR and are skipped.
+// raise DEV_ERR_CSR and are skipped.  Global reads take two dependent rounds:
+// every sub-block's row range (lanes 0..nsub-1) together with nnz, then the
+// columns of each distinct CSR row once, for all the sub-blocks that share it.
 __device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int last, uint32_t* map,
                                uint32_t* list) {
   const int lane = threadIdx.x & 31;
   for (int J = lane; J <= last; J += 32) map[J] = 0;
-  __syncwarp();
+  int qb_l = -1, lo_l = 0, hi_l = 0;
+  if (lane < nsub && row0 + lane * 64 < a.T) {
+    qb_l = (row0 + lane * 64) / a.block;
+    if (qb_l < a.nqb) {
+      lo_l = a.row_ptr[qb_l];
+      hi_l = a.row_ptr[qb_l + 1];
+    } else {
+      raise_error(a.st.err, DEV_ERR_CSR);
+      qb_l = -1;
+    }
+  }
   const int nnz = a.row_ptr[a.nqb];
+  if (qb_l >= 0 && (lo_l < 0 || hi_l < lo_l || hi_l > nnz)) {
+    raise_error(a.st.err, DEV_ERR_CSR);
+    qb_l = -1;
+  }
+  __syncwarp();
   for (int qs = 0; qs < nsub; ++qs) {
-    const int row = row0 + qs * 64;
-    if (row >= a.T) break;
-    const int qb = row / a.block;
-    if (qb >= a.nqb) {
-      if (lane == 0) raise_error(a.st.err, DEV_ERR_CSR);
-      break;
-    }
-    int lo = a.row_ptr[qb], hi = a.row_ptr[qb + 1];
-    if (lo < 0 || hi < lo || hi > nnz) {
-      if (lane == 0) raise_error(a.st.err, DEV_ERR_CSR);
-      continue;
-    }
+    const int qb = __shfl_sync(0xffffffffu, qb_l, qs);
+    if (qb < 0 || (qs > 0 && __shfl_sync(0xffffffffu, qb_l, qs - 1) == qb)) continue;
+    // Key sub-block bits of every query sub-block that reads CSR row qb.
+    uint32_t bits_even = 0;
+    for (int q2 = qs; q2 < nsub; ++q2)
+      if (__shfl_sync(0xffffffffu, qb_l, q2) == qb) bits_even |= 1u << (q2 * 2);
+    const int lo = __shfl_sync(0xffffffffu, lo_l, qs), hi = __shfl_sync(0xffffffffu, hi_l, qs);
     for (int e = lo + lane; e < hi; e += 32) {
       const int j = a.col[e];
       if (j < 0 || j >= a.nkb) {
@@ -121,7 +133,7 @@ __device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int las
       for (int ks = k0 >> 6; ks < (k1 + 63) >> 6; ++ks) {                 // 64-column sub-blocks
         const int J = ks >> 1;
         if (J > last) break;
-        atomicOr(&map[J], 1u << (qs * 2 + (ks & 1)));
+        atomicOr(&map[J], bits_even << (ks & 1));
       }
     }
   }
