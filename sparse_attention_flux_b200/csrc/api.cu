@@ -268,11 +268,12 @@ int flux_attn_prefill(flux_ctx* c, const uint16_t* q, const uint16_t* k, const u
   }
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: tensors must be 16-byte aligned");
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   int rc;
   if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
   if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
   if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&to, o, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
   flux::PrefillLaunch p;
   p.B = B;
   p.T = T;
@@ -292,7 +293,7 @@ int flux_attn_prefill(flux_ctx* c, const uint16_t* q, const uint16_t* k, const u
   p.head_mode = nullptr;
   p.blend_score = nullptr;
   p.st = status_of(c);
-  const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = flux::launch_prefill(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill: launch");
 }
 
@@ -312,10 +313,11 @@ int flux_attn_prefill_soft(flux_ctx* c, const uint16_t* q, const uint16_t* k, co
   int rc = flux_attn_prefill(c, q, k, v, o, nullptr, B, T, Hq, Hkv, d, nullptr, 0, row_ptr, col,
                              nqb, block, scale, stream);
   if (rc != FLUX_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
   if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
   if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&to, o, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
   flux::PrefillLaunch p;
   p.B = B;
   p.T = T;
@@ -335,7 +337,7 @@ int flux_attn_prefill_soft(flux_ctx* c, const uint16_t* q, const uint16_t* k, co
   p.head_mode = nullptr;
   p.blend_score = score;
   p.st = status_of(c);
-  const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = flux::launch_prefill(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill_soft: launch");
 }
 
@@ -652,11 +654,12 @@ extern "C" int flux_attn_prefill_heads(flux_ctx* c, const uint16_t* q, const uin
     return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: scale must be finite and positive");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: tensors must be 16-byte aligned");
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   int rc;
   if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
   if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
   if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&to, o, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
   flux::PrefillLaunch p;
   p.B = B;
   p.T = T;
@@ -676,7 +679,7 @@ extern "C" int flux_attn_prefill_heads(flux_ctx* c, const uint16_t* q, const uin
   p.head_mode = head_mode;
   p.blend_score = nullptr;
   p.st = status_of(c);
-  const cudaError_t e = flux::launch_prefill(tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = flux::launch_prefill(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill_heads: launch");
 }
 

@@ -32,7 +32,7 @@ struct PrefillLaunch {
 };
 int prefill_smem_bytes(int d);
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const PrefillLaunch& p, cudaStream_t stream);
+                           const CUtensorMap& to, const PrefillLaunch& p, cudaStream_t stream);
 
 struct DecodeLaunch {
   int B, Hq, Hkv, d, S_max;

@@ -153,7 +153,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+                   const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_o, const PrefillArgs a) {
   using L = Smem<D>;
   constexpr int CH = L::CH;
   constexpr uint32_t kTmemCols = 512;
@@ -414,11 +415,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const size_t row_elem = ((static_cast<size_t>(b) * a.T + t_row) * a.Hq + h) * D;
     const bool valid = t_row < a.T;
-    if (n > 0 && ok && mbar_wait(&bars[B_OD], 0, a.st)) {
+    // One decision per warpgroup (a named barrier below needs all 128 threads).
+    const bool mine = n > 0 && ok && mbar_wait(&bars[B_OD], 0, a.st);
+    const bool have_o = named_bar_and(1 + i, 128, mine);
+    if (have_o && !a.blend_score) {
+      // O_i / l -> bf16 rows staged in Q_i's (now free: every MMA has completed)
+      // shared memory in the 128-byte swizzled box layout, then stored by TMA:
+      // one 16-byte chunk per st.shared, conflict-free, no strided global stores.
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const uint32_t stage = smem_u32(sQ) + i * CH * kChunkBytes + r * 128;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + c * 32, v);
+        tmem_wait_ld();
+        const uint32_t box = stage + (c >> 1) * kChunkBytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t k16 = static_cast<uint32_t>((c & 1) * 4 + u);
+          st_shared_v4(box + ((k16 ^ static_cast<uint32_t>(r & 7)) << 4),
+                       pack_bf16x2(__uint_as_float(v[u * 8 + 0]) * inv, __uint_as_float(v[u * 8 + 1]) * inv),
+                       pack_bf16x2(__uint_as_float(v[u * 8 + 2]) * inv, __uint_as_float(v[u * 8 + 3]) * inv),
+                       pack_bf16x2(__uint_as_float(v[u * 8 + 4]) * inv, __uint_as_float(v[u * 8 + 5]) * inv),
+                       pack_bf16x2(__uint_as_float(v[u * 8 + 6]) * inv, __uint_as_float(v[u * 8 + 7]) * inv));
+        }
+      }
+      if (valid && a.lse) {
+        a.lse[(static_cast<size_t>(b) * a.Hq + h) * a.T + t_row] =
+            l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1 + i, 128);
+      const int tile_row = row0 + i * row_step;
+      if (r == 0 && tile_row < a.T) {
+        // Rows past T are clipped by the tensor map; the CTA's smem stays valid
+        // until the copy has read it.
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+          tma_store_4d(&tm_o, sQ + (i * CH + c) * kChunkBytes, c * 64, h, tile_row, b);
+        bulk_commit_group();
+        bulk_wait_read0();
+      }
+    } else if (have_o) {
       // Soft routing: blend with the row already in o (the other path's output).
-      const float r = a.blend_score ? a.blend_score[a.layer] : 0.f;
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float rb = a.blend_score[a.layer];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
@@ -426,29 +469,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(a.o + row_elem + c * 32);
-          if (a.blend_score) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const uint4 prev = dst[u];
-              const uint32_t pw[4] = {prev.x, prev.y, prev.z, prev.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                v[u * 8 + 2 * e] = __float_as_uint(
-                    fmaf(r, bf16lo_to_f32(pw[e]), (1.f - r) * __uint_as_float(v[u * 8 + 2 * e]) * inv));
-                v[u * 8 + 2 * e + 1] = __float_as_uint(
-                    fmaf(r, bf16hi_to_f32(pw[e]), (1.f - r) * __uint_as_float(v[u * 8 + 2 * e + 1]) * inv));
-              }
-            }
-          }
-          const float sc = a.blend_score ? 1.f : inv;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(v[u * 8 + 0]) * sc, __uint_as_float(v[u * 8 + 1]) * sc);
-            w.y = pack_bf16x2(__uint_as_float(v[u * 8 + 2]) * sc, __uint_as_float(v[u * 8 + 3]) * sc);
-            w.z = pack_bf16x2(__uint_as_float(v[u * 8 + 4]) * sc, __uint_as_float(v[u * 8 + 5]) * sc);
-            w.w = pack_bf16x2(__uint_as_float(v[u * 8 + 6]) * sc, __uint_as_float(v[u * 8 + 7]) * sc);
-            dst[u] = w;
+            const uint4 prev = dst[u];
+            const uint32_t pw[4] = {prev.x, prev.y, prev.z, prev.w};
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16x2(
+                  fmaf(rb, bf16lo_to_f32(pw[e]), (1.f - rb) * __uint_as_float(v[u * 8 + 2 * e]) * inv),
+                  fmaf(rb, bf16hi_to_f32(pw[e]),
+                       (1.f - rb) * __uint_as_float(v[u * 8 + 2 * e + 1]) * inv));
+            dst[u] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
@@ -459,15 +491,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (valid) {
       // No visible key (or an aborted tile): this pass contributes zero.
       uint4* dst = reinterpret_cast<uint4*>(a.o + row_elem);
-      const float r = a.blend_score ? a.blend_score[a.layer] : 0.f;
+      const float rb = a.blend_score ? a.blend_score[a.layer] : 0.f;
       for (int u = 0; u < D / 8; ++u) {
         uint4 w = make_uint4(0, 0, 0, 0);
         if (a.blend_score) {
           const uint4 prev = dst[u];
-          w.x = pack_bf16x2(r * bf16lo_to_f32(prev.x), r * bf16hi_to_f32(prev.x));
-          w.y = pack_bf16x2(r * bf16lo_to_f32(prev.y), r * bf16hi_to_f32(prev.y));
-          w.z = pack_bf16x2(r * bf16lo_to_f32(prev.z), r * bf16hi_to_f32(prev.z));
-          w.w = pack_bf16x2(r * bf16lo_to_f32(prev.w), r * bf16hi_to_f32(prev.w));
+          w.x = pack_bf16x2(rb * bf16lo_to_f32(prev.x), rb * bf16hi_to_f32(prev.x));
+          w.y = pack_bf16x2(rb * bf16lo_to_f32(prev.y), rb * bf16hi_to_f32(prev.y));
+          w.z = pack_bf16x2(rb * bf16lo_to_f32(prev.z), rb * bf16hi_to_f32(prev.z));
+          w.w = pack_bf16x2(rb * bf16lo_to_f32(prev.w), rb * bf16hi_to_f32(prev.w));
         }
         dst[u] = w;
       }
@@ -486,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 int prefill_smem_bytes(int d) { return d == 64 ? Smem<64>::ALLOC : Smem<128>::ALLOC; }
 
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const PrefillLaunch& p, cudaStream_t stream) {
+                           const CUtensorMap& to, const PrefillLaunch& p, cudaStream_t stream) {
   PrefillArgs a;
   a.B = p.B;
   a.T = p.T;
@@ -515,11 +547,11 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   if (p.d == 64) {
     const int smem = Smem<64>::ALLOC;
     cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    prefill_kernel<64><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a);
+    prefill_kernel<64><<<grid, kThreads, smem, stream>>>(tq, tk, tv, to, a);
   } else {
     const int smem = Smem<128>::ALLOC;
     cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    prefill_kernel<128><<<grid, kThreads, smem, stream>>>(tq, tk, tv, a);
+    prefill_kernel<128><<<grid, kThreads, smem, stream>>>(tq, tk, tv, to, a);
   }
   return cudaGetLastError();
 }
