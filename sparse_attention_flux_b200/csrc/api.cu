@@ -170,7 +170,8 @@ int flux_ctx_check(flux_ctx* c, flux_stream_t stream) {
     case flux::DEV_ERR_SEQLEN:
       return fail(FLUX_ERR_DEVICE_CHECK, "seqlens entry outside [0, S_max]");
     case flux::DEV_ERR_CSR:
-      return fail(FLUX_ERR_DEVICE_CHECK, "block-index list entry out of range");
+      return fail(FLUX_ERR_DEVICE_CHECK,
+                  "block-index list entry out of range or a row not strictly ascending");
     case flux::DEV_ERR_CAPACITY:
       return fail(FLUX_ERR_DEVICE_CHECK, "block-index nnz exceeds the col capacity");
     default:

@@ -85,18 +85,64 @@ struct Smem {
   static constexpr int ALLOC = TOTAL + 1024;  // room to align the base to 1024
 };
 
+// Inclusive warp prefix sum.
+__device__ __forceinline__ int warp_inclusive_sum(int x) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x;
+}
+
 // SA: the CTA's key tiles and, per tile, which (64-row query sub-block,
 // 64-column key sub-block) pairs the block mask keeps: bit (qs * 2 + ks).
-// One warp: OR every kept block of the CSR rows that the CTA's nsub 64-row
-// sub-blocks (from row0) fall in into a per-tile map, then compact it in
-// ascending tile order.  Returns the list length.  Tiles past the last tile
-// index `last` (the diagonal) are dropped (causal); CSR entries out of range
-// raise DEV_ERR_CSR and are skipped.  Global reads take two dependent rounds:
-// every sub-block's row range (lanes 0..nsub-1) together with nnz, then the
-// columns of each distinct CSR row once, for all the sub-blocks that share it.
+// One warp builds it; returns the list length.  Tiles past the last tile index
+// `last` (the diagonal) are dropped (causal).  CSR entries out of range, or a
+// row whose columns are not strictly ascending, raise DEV_ERR_CSR and are
+// skipped.
+//   Direct path -- blocks are whole key tiles (block a multiple of 128) and the
+//   unit's rows all lie in one CSR row (e.g. a head-pair unit at block 128):
+//   the row's ascending columns are the list, every tile with all bits set.
+//   Two dependent global-read rounds (the row range and nnz, then the columns).
+//   Map path otherwise: OR every kept block of the CSR rows of the nsub 64-row
+//   sub-blocks (from row0) into a per-tile map, then compact it in ascending
+//   tile order; the columns of each distinct CSR row are read once.
 __device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int last, uint32_t* map,
                                uint32_t* list) {
   const int lane = threadIdx.x & 31;
+  const int r_last = min(row0 + nsub * 64, a.T) - 1;
+  if (a.block % kBN == 0 && row0 / a.block == r_last / a.block) {
+    const int qb = row0 / a.block;
+    if (qb >= a.nqb) {
+      if (lane == 0) raise_error(a.st.err, DEV_ERR_CSR);
+      return 0;
+    }
+    const int lo = a.row_ptr[qb], hi = a.row_ptr[qb + 1], nnz = a.row_ptr[a.nqb];
+    if (lo < 0 || hi < lo || hi > nnz) {
+      if (lane == 0) raise_error(a.st.err, DEV_ERR_CSR);
+      return 0;
+    }
+    const int tpb = a.block / kBN;                          // key tiles per block
+    const uint32_t full = ((1u << (2 * nsub)) - 1u) << 24;  // every (qs, ks) bit
+    int n = 0, prev = -1;
+    for (int base = lo; base < hi; base += 32) {
+      const int e = base + lane;
+      const int j = e < hi ? a.col[e] : 0;
+      const int jp = __shfl_up_sync(0xffffffffu, j, 1);
+      const int before = lane == 0 ? prev : jp;
+      const bool ok = e < hi && j >= 0 && j < a.nkb && j > before;
+      if (e < hi && !ok) raise_error(a.st.err, DEV_ERR_CSR);
+      const int cnt = ok ? max(0, min(tpb, last - j * tpb + 1)) : 0;
+      const int incl = warp_inclusive_sum(cnt);
+      for (int t = 0; t < cnt; ++t)
+        list[n + incl - cnt + t] = static_cast<uint32_t>(j * tpb + t) | full;
+      n += __shfl_sync(0xffffffffu, incl, 31);
+      prev = __shfl_sync(0xffffffffu, j, min(31, hi - 1 - base));
+    }
+    return n;
+  }
   for (int J = lane; J <= last; J += 32) map[J] = 0;
   int qb_l = -1, lo_l = 0, hi_l = 0;
   if (lane < nsub && row0 + lane * 64 < a.T) {
@@ -123,9 +169,15 @@ __device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int las
     for (int q2 = qs; q2 < nsub; ++q2)
       if (__shfl_sync(0xffffffffu, qb_l, q2) == qb) bits_even |= 1u << (q2 * 2);
     const int lo = __shfl_sync(0xffffffffu, lo_l, qs), hi = __shfl_sync(0xffffffffu, hi_l, qs);
-    for (int e = lo + lane; e < hi; e += 32) {
-      const int j = a.col[e];
-      if (j < 0 || j >= a.nkb) {
+    int prev = -1;
+    for (int base = lo; base < hi; base += 32) {
+      const int e = base + lane;
+      const int j = e < hi ? a.col[e] : 0;
+      const int jp = __shfl_up_sync(0xffffffffu, j, 1);
+      const int before = lane == 0 ? prev : jp;
+      prev = __shfl_sync(0xffffffffu, j, min(31, hi - 1 - base));
+      if (e >= hi) continue;
+      if (j < 0 || j >= a.nkb || j <= before) {
         raise_error(a.st.err, DEV_ERR_CSR);
         continue;
       }

@@ -158,3 +158,71 @@ def test_qwen3_4b_layer_prefill_sampled_rows(ctx, mode):
         for (h, r, pos) in needles:
             target = V[0, pos, h // (Hq // Hkv)].mean(0)
             assert np.abs(synth.bf16_bits_to_f32(o[0, r, h]) - target).max() < 0.1
+
+
+def _random_causal_block_mask(nb, keep, seed):
+    r = np.random.default_rng(seed)
+    m = (r.random((nb, nb)) < keep).astype(np.uint8)
+    m[np.arange(nb), np.arange(nb)] = 1          # every row keeps its diagonal block
+    return np.tril(m)
+
+
+@pytest.mark.parametrize("case", [  # B, T, Hq, Hkv, d, block
+    (1, 1000, 8, 2, 128, 128),      # head pairs, direct list (one CSR row per unit)
+    (1, 1000, 4, 4, 128, 128),      # row pairs (G = 1): union of two CSR rows
+    (1, 1100, 8, 2, 128, 256),      # head pairs, two key tiles per block
+    (2, 900, 6, 6, 64, 256),        # row pairs inside one 256-row block: direct list
+    (1, 700, 4, 1, 128, 64),        # block 64: per-64 sub-block masks
+])
+def test_random_block_mask_matches_oracle(ctx, case):
+    """Arbitrary kept-block sets (not only sink + window), through the CSR list."""
+    B, T, Hq, Hkv, d, block = case
+    q, k, v = synth.attention_inputs(B, T, Hq, Hkv, d, seed=77 + T + block)
+    nb = (T + block - 1) // block
+    mask = _random_causal_block_mask(nb, 0.35, seed=T + block)
+    dev = ctx.device
+    m_t = torch.from_numpy(mask).to(dev)
+    rp = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(nb * nb, dtype=torch.int32, device=dev)
+    ctx.build_block_index(m_t, rp, col)
+    qt, kt, vt = (synth.torch_from_bits(x).to(dev) for x in (q, k, v))
+    o = torch.full_like(qt, float("nan"))
+    lm = torch.zeros(1, dtype=torch.uint8, device=dev)
+    ctx.attn_prefill(qt, kt, vt, o, 1 / np.sqrt(d), layer_mode=lm, row_ptr=rp, col=col,
+                     block=block)
+    ctx.check()
+    ro, _ = oracle.attn_prefill(q, k, v, 1 / np.sqrt(d), block_mask=mask, block=block)
+    assert_close_attn(bits_of(o), ro, f"random mask {case}")
+
+
+@pytest.mark.parametrize("block", [128, 64])
+@pytest.mark.parametrize("bad", ["out_of_range", "descending", "repeat"])
+def test_malformed_csr_is_a_device_error(ctx, block, bad):
+    """A CSR row out of range, out of order or with a repeated column is reported
+    (FLUX_ERR_DEVICE_CHECK) and the context keeps working."""
+    from sparse_attention_flux_b200.flux import FLUX_ERR_DEVICE_CHECK
+    B, T, Hq, Hkv, d = 1, 512, 4, 2, 128
+    nb = T // block
+    q, k, v = synth.attention_inputs(B, T, Hq, Hkv, d, seed=3)
+    dev = ctx.device
+    qt, kt, vt = (synth.torch_from_bits(x).to(dev) for x in (q, k, v))
+    o = torch.empty_like(qt)
+    rows = [list(range(i + 1)) for i in range(nb)]       # causal, all blocks kept
+    last = rows[-1]
+    if bad == "out_of_range":
+        last[1] = nb + 3
+    elif bad == "descending":
+        last[0], last[1] = last[1], last[0]
+    else:
+        last[1] = last[0]
+    rp = torch.tensor(np.cumsum([0] + [len(r) for r in rows]), dtype=torch.int32, device=dev)
+    col = torch.tensor([c for r in rows for c in r], dtype=torch.int32, device=dev)
+    lm = torch.zeros(1, dtype=torch.uint8, device=dev)
+    ctx.attn_prefill(qt, kt, vt, o, 0.1, layer_mode=lm, row_ptr=rp, col=col, block=block)
+    with pytest.raises(FluxError) as e:
+        ctx.check()
+    assert e.value.code == FLUX_ERR_DEVICE_CHECK
+    # the context is still usable: a well-formed call gives the oracle's answer
+    o_ok, _ = _run(ctx, q, k, v, 0.1, 0, block, 1, 2)
+    ro, _ = _oracle(q, k, v, 0.1, True, block, 1, 2)
+    assert_close_attn(o_ok, ro, "after malformed CSR")
