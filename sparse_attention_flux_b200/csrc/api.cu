@@ -459,6 +459,7 @@ int flux_attn_decode_sa_compact(flux_ctx* c, const uint16_t* q, const uint16_t* 
   flux::DecodeLaunch p;
   flux::decode_plan(B, Hkv, rows, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
                     &p.chunk_fa, &p.tiles_sa);
+  p.nsplit = flux::decode_sa_splits(sink_blocks, window_blocks, block, p.tiles_sa);  // SA only
   const size_t nrow = static_cast<size_t>(B) * Hq * p.nsplit;
   const size_t o_bytes = align256(nrow * d * sizeof(float));
   if (o_bytes + align256(nrow * 2 * sizeof(float)) > c->workspace_bytes)

@@ -434,6 +434,13 @@ void decode_plan(int B, int Hkv, int S_max, int sink_blocks, int window_blocks, 
   *tiles_sa = static_cast<int>(tsa);
 }
 
+int decode_sa_splits(int sink_blocks, int window_blocks, int block, int tiles_sa) {
+  const long long sa_tiles = (static_cast<long long>(sink_blocks) * block + kTok - 1) / kTok +
+                             (static_cast<long long>(window_blocks) * block + kTok - 1) / kTok;
+  const long long t = tiles_sa > 0 ? tiles_sa : 1;
+  return static_cast<int>(std::max<long long>(1, (sa_tiles + t - 1) / t));
+}
+
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int nsplit) {
   const size_t rows = static_cast<size_t>(B) * Hq * nsplit;
   size_t bytes = rows * d * sizeof(float);

@@ -55,6 +55,8 @@ struct DecodeLaunch {
 // Split plan for a shape (host only): number of splits and chunk lengths.
 void decode_plan(int B, int Hkv, int S_max, int sink_blocks, int window_blocks, int block,
                  int num_sms, int* nsplit, int* chunk_fa, int* tiles_sa);
+// Active splits of an SA-only (compact ring) launch: its grid needs no FA splits.
+int decode_sa_splits(int sink_blocks, int window_blocks, int block, int tiles_sa);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int nsplit);
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeLaunch& p,
                           cudaStream_t stream);
