@@ -33,6 +33,7 @@ a bounded sample of the same workload, as the reference arm.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -81,6 +82,26 @@ def sa_decode_tokens(s, block, sink, W):
     nbs = -(-s // block)
     win_start = max(n_sink, max(0, nbs - W) * block)
     return n_sink + (s - win_start)
+
+
+def recorded_traffic(key):
+    """DRAM bytes per launch (read + write) of a kernel from its ncu capture, recorded in
+    profiles/dram_traffic.json together with a SHA-256 of the sources it was built from;
+    None when there is no record or any of those sources has changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(key)
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for rel in rec["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
+    return int(rec["bytes_per_launch"])
 
 
 def load_peaks():
@@ -765,7 +786,8 @@ def run_flux(args, rank, world, dev_index):
         }
         roof_dec = {"bound": "hbm", "achieved": round(fa_dec_gbs, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4),
-                    "traffic": None, "kernel": "decode_kernel<128,4> (FA layer, incl. its append)"}
+                    "traffic": recorded_traffic("decode_fa_B16_S131072"),
+                    "kernel": "decode_kernel<128,4> (FA layer, incl. its append)"}
         dec["roofline"] = roof_dec
         dec["routing_granularity"] = dw.granularity(8)
         dec["sa_layer"] = dw.sa_layer(10)
@@ -791,7 +813,8 @@ def run_flux(args, rank, world, dev_index):
                    "l2": "inputs larger than L2 (640 MB prefill, 17 GB decode KV); no flush",
                    "parallelism": f"replicas x{world} (no exchange)"},
         "roofline": {"bound": "tensor", "achieved": round(fa_tflops, 1), "peak": peak_t,
-                     "unit": "TFLOP/s", "frac": round(fa_tflops / peak_t, 4), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(fa_tflops / peak_t, 4),
+                     "traffic": recorded_traffic("prefill_fa_T32768"),
                      "kernel": "prefill_kernel<128> (FA layer)",
                      "peak_source": f"{peak_src} bf16_tflops_sustained"},
         "sa_prefill": {"TFLOP/s": round(sa_tflops, 1), "ms": round(sa_avg, 4),
