@@ -152,9 +152,11 @@ int flux_build_block_index(flux_ctx* ctx, const uint8_t* block_mask, int nqb, in
  *   row_ptr/col: the CSR list from flux_build_block_index over nqb >=
  *   ceil(T / block) q-blocks; required unless layer_mode == NULL.  Each row's
  *   columns must be strictly ascending and < ceil(T / block), as
- *   flux_build_block_index writes them; an entry out of range or out of order
- *   is a device-checked error (FLUX_ERR_DEVICE_CHECK from flux_ctx_check) and
- *   is skipped.
+ *   flux_build_block_index writes them.  A row range or an entry out of range,
+ *   or a row out of order, is a device-checked error (FLUX_ERR_DEVICE_CHECK from
+ *   flux_ctx_check): the query rows whose key list reads that CSR row (that
+ *   q-block's rows, up to the 256-row unit holding them) are written as zero,
+ *   lse -inf.
  *   block: 64 or a multiple of 128.  d: 64 or 128.  With layer_mode given,
  *   T <= 262144 (the CTA's key-tile list lives in shared memory).  scale: score scale
  *   (1/sqrt(d) for the models on the pages).

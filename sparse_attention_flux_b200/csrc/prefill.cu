@@ -99,9 +99,9 @@ __device__ __forceinline__ int warp_inclusive_sum(int x) {
 // SA: the CTA's key tiles and, per tile, which (64-row query sub-block,
 // 64-column key sub-block) pairs the block mask keeps: bit (qs * 2 + ks).
 // One warp builds it; returns the list length.  Tiles past the last tile index
-// `last` (the diagonal) are dropped (causal).  CSR entries out of range, or a
-// row whose columns are not strictly ascending, raise DEV_ERR_CSR and are
-// skipped.
+// `last` (the diagonal) are dropped (causal).  A CSR row out of range, an entry
+// out of range or a row whose columns are not strictly ascending raises
+// DEV_ERR_CSR and empties the list, so the unit's rows are written as zero.
 //   Direct path -- blocks are whole key tiles (block a multiple of 128) and the
 //   unit's rows all lie in one CSR row (e.g. a head-pair unit at block 128):
 //   the row's ascending columns are the list, every tile with all bits set.
@@ -133,7 +133,10 @@ __device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int las
       const int jp = __shfl_up_sync(0xffffffffu, j, 1);
       const int before = lane == 0 ? prev : jp;
       const bool ok = e < hi && j >= 0 && j < a.nkb && j > before;
-      if (e < hi && !ok) raise_error(a.st.err, DEV_ERR_CSR);
+      if (__any_sync(0xffffffffu, e < hi && !ok)) {
+        if (lane == 0) raise_error(a.st.err, DEV_ERR_CSR);
+        return 0;
+      }
       const int cnt = ok ? max(0, min(tpb, last - j * tpb + 1)) : 0;
       const int incl = warp_inclusive_sum(cnt);
       for (int t = 0; t < cnt; ++t)
@@ -151,15 +154,12 @@ __device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int las
       lo_l = a.row_ptr[qb_l];
       hi_l = a.row_ptr[qb_l + 1];
     } else {
-      raise_error(a.st.err, DEV_ERR_CSR);
-      qb_l = -1;
+      qb_l = -2;   // row out of range
     }
   }
   const int nnz = a.row_ptr[a.nqb];
-  if (qb_l >= 0 && (lo_l < 0 || hi_l < lo_l || hi_l > nnz)) {
-    raise_error(a.st.err, DEV_ERR_CSR);
-    qb_l = -1;
-  }
+  if (qb_l >= 0 && (lo_l < 0 || hi_l < lo_l || hi_l > nnz)) qb_l = -2;
+  bool bad = __any_sync(0xffffffffu, qb_l == -2);
   __syncwarp();
   for (int qs = 0; qs < nsub; ++qs) {
     const int qb = __shfl_sync(0xffffffffu, qb_l, qs);
@@ -178,7 +178,7 @@ __device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int las
       prev = __shfl_sync(0xffffffffu, j, min(31, hi - 1 - base));
       if (e >= hi) continue;
       if (j < 0 || j >= a.nkb || j <= before) {
-        raise_error(a.st.err, DEV_ERR_CSR);
+        bad = true;
         continue;
       }
       const int k0 = j * a.block, k1 = min((j + 1) * a.block, a.T);   // key range of block j
@@ -188,6 +188,10 @@ __device__ int build_tile_list(const PrefillArgs& a, int row0, int nsub, int las
         atomicOr(&map[J], bits_even << (ks & 1));
       }
     }
+  }
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) raise_error(a.st.err, DEV_ERR_CSR);
+    return 0;
   }
   __syncwarp();
   int n = 0;

@@ -222,6 +222,10 @@ def test_malformed_csr_is_a_device_error(ctx, block, bad):
     with pytest.raises(FluxError) as e:
         ctx.check()
     assert e.value.code == FLUX_ERR_DEVICE_CHECK
+    # the rows that read the malformed CSR row are zeroed, the others computed
+    o_b = bits_of(o)
+    assert np.all(o_b[:, (nb - 1) * block:] == 0)
+    assert np.any(o_b[:, :block] != 0)
     # the context is still usable: a well-formed call gives the oracle's answer
     o_ok, _ = _run(ctx, q, k, v, 0.1, 0, block, 1, 2)
     ro, _ = _oracle(q, k, v, 0.1, True, block, 1, 2)
