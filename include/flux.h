@@ -283,7 +283,7 @@ int flux_attn_decode_heads(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_c
  *   wait ran out); NULL to skip.
  *   Limits: B * Hkv <= 4096 and B * Hq * nsplit * (d + 2) * 4 bytes of
  *   partials within the 32 MiB (nsplit as flux_decode_workspace_bytes plans
- *   it; e.g. B 16, Hq 32, d 128 at 131072 tokens needs 17 MiB).  Larger shapes
+ *   it; e.g. B 16, Hq 32, d 128 at 131072 tokens takes 4 splits, 1.1 MiB).  Larger shapes
  *   return FLUX_ERR_SHAPE before any device work.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
