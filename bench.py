@@ -676,7 +676,7 @@ def run_flux(args, rank, world, dev_index):
 
     # e2e: host buffers in and out through the same public API, copies inside the timed
     # region -- pipelined over three streams, and serial for reference.
-    e2e_steps = max(4, args.steps // 2)
+    e2e_steps = max(4, args.steps)   # the same K steps as the device-timed region
     wl.e2e_pipelined(2)
     barrier()
     e2e_ms = ranks_max(wl.e2e_pipelined(e2e_steps))
@@ -830,7 +830,10 @@ def run_flux(args, rank, world, dev_index):
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                 "how": "pinned host -> device copy of Q/K/V/hidden, router + index + FA + SA "
                        "layers, device -> host copy of both outputs, every step; copies of "
-                       "steps k+1 / k-1 overlap step k's compute on separate streams",
+                       "steps k+1 / k-1 overlap step k's compute on separate streams; timed "
+                       "over K steps from the first upload to the last download (pipeline "
+                       "fill and drain included)",
+                "steps": e2e_steps,
                 "serial_ms_per_step": round(e2e_serial_ms, 4),
                 "serial_value": round(e2e_serial_value, 2)},
         "gpu_launches": launches,
