@@ -346,7 +346,7 @@ class DecodeWorkload:
                             for s in range(steps)) / steps
         n_fa = int(self.mode_h.sum())
         self.bytes_per_step = n_fa * self.bytes_fa + (DEC_LAYERS - n_fa) * self.bytes_sa
-        self.launches = 2 * DEC_LAYERS
+        self.launches = DEC_LAYERS   # one fused append + decode per layer
         self.kv_gb = (2 * 2 * DEC_B * self.S_max * HKV * D * 2 +
                       len(self.rings) * 2 * DEC_B * (SINK + WIN) * BLOCK * HKV * D * 2) / 1e9
 
@@ -435,7 +435,10 @@ class DecodeWorkload:
         self.sl_cur.copy_(self.seqlens[s], non_blocking=True)
         self.graph.replay()
 
-    def step(self, s, fa_events=None, sl=None):
+    def step(self, s, fa_events=None, sl=None, fused=True):
+        """One 36-layer decode step.  fused: flux_attn_decode_append (the step's token is
+        written into the layer's cache by the decode launch itself: 36 launches); else
+        flux_kv_write then the decode (72 launches)."""
         c = self.ctx
         fa_i = 0
         sl = self.seqlens[s] if sl is None else sl
@@ -446,15 +449,26 @@ class DecodeWorkload:
                 timed = fa_events is not None and fa_i == 1
                 if timed:
                     fa_events[0].record()
-                c.kv_write(self.new_k, self.new_v, sl, kc, vc)
-                c.attn_decode(self.q, kc, vc, sl, self.o, self.scale, layer_mode=self.mode,
-                              layer=layer, sink_blocks=SINK, window_blocks=WIN, block=BLOCK)
+                if fused:
+                    c.attn_decode_append(self.q, self.new_k, self.new_v, kc, vc, sl, self.o,
+                                         self.scale, layer_mode=self.mode, layer=layer,
+                                         sink_blocks=SINK, window_blocks=WIN, block=BLOCK)
+                else:
+                    c.kv_write(self.new_k, self.new_v, sl, kc, vc)
+                    c.attn_decode(self.q, kc, vc, sl, self.o, self.scale, layer_mode=self.mode,
+                                  layer=layer, sink_blocks=SINK, window_blocks=WIN, block=BLOCK)
                 if timed:
                     fa_events[1].record()
             else:
                 kr, vr = self.rings[layer]
-                c.kv_write(self.new_k, self.new_v, sl, kr, vr, SINK, WIN, BLOCK)
-                c.attn_decode_sa_compact(self.q, kr, vr, sl, self.o, self.scale, SINK, WIN, BLOCK)
+                if fused:
+                    c.attn_decode_append(self.q, self.new_k, self.new_v, kr, vr, sl, self.o,
+                                         self.scale, sink_blocks=SINK, window_blocks=WIN,
+                                         block=BLOCK, compact=True)
+                else:
+                    c.kv_write(self.new_k, self.new_v, sl, kr, vr, SINK, WIN, BLOCK)
+                    c.attn_decode_sa_compact(self.q, kr, vr, sl, self.o, self.scale, SINK, WIN,
+                                             BLOCK)
 
 
 def _events(torch, n):
@@ -755,6 +769,14 @@ def run_flux(args, rank, world, dev_index):
         e1.synchronize()
         fa_dec_ms = [a_.elapsed_time(b_) for a_, b_ in fevs]
         eager_ms = e0.elapsed_time(e1) / dw.steps
+        # the same steps with the append as its own launch (flux_kv_write), for comparison
+        n_sep = min(8, dw.steps)
+        e0.record()
+        for s in range(n_sep):
+            dw.step(s, fused=False)
+        e1.record()
+        e1.synchronize()
+        separate_ms = e0.elapsed_time(e1) / n_sep
         ctx.check()
         # timed: the same steps replayed from a CUDA graph
         dw.capture()
@@ -774,12 +796,14 @@ def run_flux(args, rank, world, dev_index):
         fa_dec_gbs = dw.bytes_fa / (fa_dec_avg * 1e-3) / 1e9
         dec = {
             "workload": "qwen3-4b-36L-routed-decode: B 16, KV 131072+step, 18 FA (full cache) / "
-                        f"18 SA (ring of sink 1 + 16 blocks), append + decode per layer, {dw.steps} steps",
+                        f"18 SA (ring of sink 1 + 16 blocks), fused append + decode per layer, {dw.steps} steps",
             "kv_resident_gb": round(dw.kv_gb, 2),
             "value": round(dec_gbs, 1), "unit": "GB/s (KV bytes that must be read)",
             "ms_per_step": round(dec_ms, 4), "gpu_launches_per_step": dw.launches,
-            "launch": "CUDA graph of one 36-layer step (72 launches), seqlens updated per replay",
+            "launch": "CUDA graph of one 36-layer step (36 fused append + decode launches), "
+                      "seqlens updated per replay",
             "eager_ms_per_step": round(eager_ms, 4),
+            "separate_append_eager_ms_per_step": round(separate_ms, 4),
             "frac_of_hbm": round(dec_gbs / peaks["hbm_gbs"], 4),
             "fa_layer": {"GB/s": round(fa_dec_gbs, 1), "ms": round(fa_dec_avg, 4),
                          "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4)},

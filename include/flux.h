@@ -17,6 +17,7 @@
  *   flux_attn_decode           one layer, one new token per sequence
  *   flux_kv_write              append / fill a full cache or an SA layer's ring
  *   flux_attn_decode_sa_compact  SA decode over the ring (sink + last W blocks)
+ *   flux_attn_decode_append    append the step's token + decode, one launch
  *
  * Conventions shared by every entry point
  *   - Every tensor pointer is a DEVICE pointer owned by the caller; the
@@ -241,6 +242,29 @@ int flux_attn_decode_sa_compact(flux_ctx* ctx, const uint16_t* q, const uint16_t
                                 uint16_t* o, float* lse, int B, int Hq, int Hkv, int d,
                                 int sink_blocks, int window_blocks, int block, float scale,
                                 flux_stream_t stream);
+
+/* flux_attn_decode_append: one decode step of one layer with the step's KV
+ * append fused in (same section of the gist.science summary: the new token's
+ * K/V enters the layer's cache, then the query attends).  k_new/v_new
+ * [B, Hkv, d] bf16 are the new token's rows; seqlens[b] = s counts it (the new
+ * token is token s - 1).  The decode CTA whose split reads token s - 1 writes
+ * the rows into the cache first, so the result equals flux_kv_write (n_src 1)
+ * followed by the decode, in one launch:
+ *   compact == 0: k_cache/v_cache is a full cache [B, cache_rows, Hkv, d]
+ *     (cache_rows = S_max, s <= S_max), routed by layer_mode[layer] exactly as
+ *     flux_attn_decode (layer_mode NULL = FA);
+ *   compact == 1: it is an SA layer's ring, cache_rows = (sink_blocks +
+ *     window_blocks) * block, block a multiple of 64, as
+ *     flux_attn_decode_sa_compact; layer_mode is ignored.
+ * A seqlens entry below 1 (no token to append) or above S_max for a full cache
+ * is a device-checked error: nothing is written for that sequence and its
+ * output is zero.  Other limits and the workspace as flux_attn_decode. */
+int flux_attn_decode_append(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_new,
+                            const uint16_t* v_new, uint16_t* k_cache, uint16_t* v_cache,
+                            int cache_rows, const int32_t* seqlens, uint16_t* o, float* lse,
+                            int B, int Hq, int Hkv, int d, const uint8_t* layer_mode, int layer,
+                            int sink_blocks, int window_blocks, int block, int compact,
+                            float scale, flux_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * Per-head routing (the contrast case).  Flux Attention routes whole layers;

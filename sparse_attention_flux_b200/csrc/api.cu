@@ -493,6 +493,78 @@ int flux_attn_decode_sa_compact(flux_ctx* c, const uint16_t* q, const uint16_t* 
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_sa_compact: launch");
 }
 
+int flux_attn_decode_append(flux_ctx* c, const uint16_t* q, const uint16_t* k_new,
+                            const uint16_t* v_new, uint16_t* k_cache, uint16_t* v_cache,
+                            int cache_rows, const int32_t* seqlens, uint16_t* o, float* lse,
+                            int B, int Hq, int Hkv, int d, const uint8_t* layer_mode, int layer,
+                            int sink_blocks, int window_blocks, int block, int compact,
+                            float scale, flux_stream_t stream) {
+  static const char* name = "flux_attn_decode_append";
+  if (!c || !q || !k_new || !v_new || !k_cache || !v_cache || !seqlens || !o)
+    return fail(FLUX_ERR_INVALID_ARG, "%s: null tensor", name);
+  if (B < 1 || Hq < 1 || Hkv < 1 || cache_rows < 1)
+    return fail(FLUX_ERR_SHAPE, "%s: sizes must be positive", name);
+  if (d != 64 && d != 128)
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: head_dim %d (supported: 64, 128)", name, d);
+  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: Hq/Hkv must be 1, 2 or 4 (%d, %d)", name, Hq, Hkv);
+  if (block < 1 || sink_blocks < 0 || window_blocks < 1 || (compact != 0 && compact != 1))
+    return fail(FLUX_ERR_INVALID_ARG, "%s: bad block / sink / window / compact", name);
+  if (compact && (block < 64 || block % 64 != 0))
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: a ring needs block a multiple of 64", name);
+  if (compact && static_cast<long long>(sink_blocks + window_blocks) * block != cache_rows)
+    return fail(FLUX_ERR_SHAPE, "%s: ring cache_rows must be (sink + window) * block", name);
+  if (!compact && layer_mode && layer < 0)
+    return fail(FLUX_ERR_INVALID_ARG, "%s: negative layer", name);
+  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "%s: scale must be finite and positive", name);
+  if (static_cast<long long>(B) * Hkv > kMaxTickets)
+    return fail(FLUX_ERR_SHAPE, "%s: B * Hkv > %d", name, kMaxTickets);
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache))
+    return fail(FLUX_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", name);
+  flux::DecodeLaunch p;
+  flux::decode_plan(B, Hkv, cache_rows, sink_blocks, window_blocks, block, c->num_sms,
+                    &p.nsplit, &p.chunk_fa, &p.tiles_sa);
+  if (compact) p.nsplit = flux::decode_sa_splits(sink_blocks, window_blocks, block, p.tiles_sa);
+  const size_t nrow = static_cast<size_t>(B) * Hq * p.nsplit;
+  const size_t o_bytes = align256(nrow * d * sizeof(float));
+  const size_t need = o_bytes + align256(nrow * 2 * sizeof(float));
+  if (need > c->workspace_bytes)
+    return fail(FLUX_ERR_SHAPE, "%s: workspace %zu < %zu bytes", name, c->workspace_bytes, need);
+  CUtensorMap tk, tv;
+  int rc;
+  if ((rc = make_map_4d(&tk, k_cache, d, Hkv, cache_rows, B, 64, 64)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, v_cache, d, Hkv, cache_rows, B, 64, 64)) != FLUX_OK) return rc;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.S_max = cache_rows;
+  p.q = q;
+  p.seqlens = seqlens;
+  p.o = o;
+  p.lse = lse;
+  p.layer_mode = compact ? nullptr : layer_mode;
+  p.layer = compact ? 0 : layer;
+  p.sink_blocks = sink_blocks;
+  p.window_blocks = window_blocks;
+  p.block = block;
+  p.scale = scale;
+  p.part_o = static_cast<float*>(c->workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
+  p.tickets = c->tickets;
+  p.compact = compact;
+  p.head_mode = nullptr;
+  p.st = status_of(c);
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_append: launch");
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

@@ -67,6 +67,16 @@ struct Range {
   int win_start, s;  // SA: window segment [win_start, s)
   int ntiles;
   int n_active;      // active splits of this (sequence, kv head)
+  // Does this split read token u?
+  __device__ __forceinline__ bool holds(int u) const {
+    if (ntiles == 0 || u < 0) return false;
+    if (fa) return start <= u && u < end;
+    int vt;
+    if (u < n_sink) vt = u / 64;
+    else if (u >= win_start && u < s) vt = t_sink + (u - win_start) / 64;
+    else return false;
+    return v0 <= vt && vt < v1;
+  }
   // Tile k of this split: tokens [*t0, *t1).
   __device__ __forceinline__ void tile(int k, int* t0, int* t1) const {
     if (fa) {
@@ -142,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     fa = !a.compact && (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
   }
   int s = a.seqlens[b];
-  if (s < 0 || (!a.compact && s > a.S_max)) {
+  if (s < 0 || (!a.compact && s > a.S_max) || (a.k_new && s < 1)) {
     if (i == 0 && g == 0 && tid == 0) raise_error(a.st.err, DEV_ERR_SEQLEN);
     s = 0;
   }
@@ -179,6 +189,27 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == kComputeWarps) {
     // ------------------------------------------------------------ producer
+    if (a.k_new && rg.holds(s - 1)) {
+      // Fused append: this split reads token s - 1, so it writes the new K/V
+      // rows into the cache (the ring slot of the token's block when compact)
+      // before any of its tiles is loaded; no other CTA reads that row.
+      const int u = s - 1;
+      int row = u;
+      if (a.compact && u >= a.sink_blocks * a.block) {
+        const int j = u / a.block;
+        row = (a.sink_blocks + j % a.window_blocks) * a.block + u % a.block;
+      }
+      const size_t dst = ((static_cast<size_t>(b) * a.S_max + row) * a.Hkv + g) * D;
+      const size_t src = (static_cast<size_t>(b) * a.Hkv + g) * D;
+      if (lane < D / 8) {
+        reinterpret_cast<uint4*>(a.k_cache + dst)[lane] =
+            reinterpret_cast<const uint4*>(a.k_new + src)[lane];
+        reinterpret_cast<uint4*>(a.v_cache + dst)[lane] =
+            reinterpret_cast<const uint4*>(a.v_new + src)[lane];
+      }
+      fence_proxy_async_global();
+      __syncwarp();
+    }
     if (lane == 0 && ntiles > 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);

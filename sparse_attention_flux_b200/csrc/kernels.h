@@ -51,6 +51,13 @@ struct DecodeLaunch {
   float* part_ml;   // [B, Hq, nsplit, 2]
   int* tickets;     // [B, Hkv], zero between calls
   DevStatus st;
+  // Fused append (null = none): the new token's K/V rows k_new/v_new [B, Hkv, d]
+  // are written into k_cache/v_cache (the tensors behind the maps) at token
+  // seqlens[b] - 1 -- its ring slot when compact -- by the CTA that reads it.
+  const uint16_t* k_new = nullptr;
+  const uint16_t* v_new = nullptr;
+  uint16_t* k_cache = nullptr;
+  uint16_t* v_cache = nullptr;
 };
 // Split plan for a shape (host only): number of splits and chunk lengths.
 void decode_plan(int B, int Hkv, int S_max, int sink_blocks, int window_blocks, int block,

@@ -70,6 +70,8 @@ _SIGNATURES = {
                                      _f, _vp], _i),
     "flux_attn_decode_noalloc": ([_vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i, _i,
                                   _i, _i, _f, _vp, _vp], _i),
+    "flux_attn_decode_append": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i,
+                                 _vp, _i, _i, _i, _i, _i, _f, _vp], _i),
 }
 
 
@@ -346,6 +348,31 @@ class Context:
                                                  _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq,
                                                  k_ring.shape[2], d, sink_blocks, window_blocks,
                                                  block, float(scale), _stream(stream)))
+
+    def attn_decode_append(self, q, k_new, v_new, k_cache, v_cache, seqlens, o, scale: float,
+                           layer_mode=None, layer: int = 0, sink_blocks: int = 1,
+                           window_blocks: int = 16, block: int = 128, compact: bool = False,
+                           lse=None, stream=None):
+        """One decode step with the step's KV append fused: k_new/v_new [B, Hkv, d] (or
+        [B, 1, Hkv, d]) become token seqlens[b] - 1 of the cache -- a full cache routed by
+        layer_mode, or (compact=True) an SA layer's ring -- and q attends."""
+        import torch
+        for n_, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                      ("v_cache", v_cache), ("o", o)):
+            _need(t, torch.bfloat16, n_, self.device)
+        _need(seqlens, torch.int32, "seqlens", self.device)
+        _need(lse, torch.float32, "lse", self.device)
+        _need(layer_mode, torch.uint8, "layer_mode", self.device)
+        B, Hq, d = q.shape
+        _, rows, Hkv, _ = k_cache.shape
+        if k_cache.shape[0] != B or k_cache.shape[3] != d or v_cache.shape != k_cache.shape \
+                or o.shape != q.shape or k_new.numel() != B * Hkv * d or v_new.shape != k_new.shape:
+            raise ValueError("q / k_new / cache / o shapes are inconsistent")
+        _check(lib().flux_attn_decode_append(self._h, _ptr(q), _ptr(k_new), _ptr(v_new),
+                                             _ptr(k_cache), _ptr(v_cache), rows, _ptr(seqlens),
+                                             _ptr(o), _ptr(lse), B, Hq, Hkv, d, _ptr(layer_mode),
+                                             layer, sink_blocks, window_blocks, block,
+                                             1 if compact else 0, float(scale), _stream(stream)))
 
 
 def attn_decode_noalloc(q, k_cache, v_cache, seqlens, o, scale: float, layer_mode=None,

@@ -13,7 +13,9 @@ from sparse_attention_flux_b200.flux import Context
 pytestmark = pytest.mark.gpu
 
 
-def test_routed_step_graph_replay_matches_eager():
+@pytest.mark.parametrize("fused", [False, True])
+def test_routed_step_graph_replay_matches_eager(fused):
+    """fused: the decodes append the step's token themselves (flux_attn_decode_append)."""
     dev = torch.device("cuda", 0)
     T, Hq, Hkv, d, blk = 1024, 8, 2, 128, 128
     B, S_max = 2, 3000
@@ -47,11 +49,18 @@ def test_routed_step_graph_replay_matches_eager():
             for layer in (0, 1):
                 ctx.attn_prefill(q, k, v, outs[layer], 1 / math.sqrt(d), layer_mode=mode,
                                  layer=layer, row_ptr=rp, col=col, block=blk)
-            ctx.kv_write(nk, nv, sl, kc, vc)
-            ctx.attn_decode(qd, kc, vc, sl, outs[2], 1 / math.sqrt(d), layer_mode=mode, layer=0,
-                            sink_blocks=1, window_blocks=16, block=blk)
-            ctx.kv_write(nk, nv, sl, kr, vr, 1, 16, blk)
-            ctx.attn_decode_sa_compact(qd, kr, vr, sl, outs[3], 1 / math.sqrt(d), 1, 16, blk)
+            if fused:
+                ctx.attn_decode_append(qd, nk, nv, kc, vc, sl, outs[2], 1 / math.sqrt(d),
+                                       layer_mode=mode, layer=0, sink_blocks=1, window_blocks=16,
+                                       block=blk)
+                ctx.attn_decode_append(qd, nk, nv, kr, vr, sl, outs[3], 1 / math.sqrt(d),
+                                       sink_blocks=1, window_blocks=16, block=blk, compact=True)
+            else:
+                ctx.kv_write(nk, nv, sl, kc, vc)
+                ctx.attn_decode(qd, kc, vc, sl, outs[2], 1 / math.sqrt(d), layer_mode=mode,
+                                layer=0, sink_blocks=1, window_blocks=16, block=blk)
+                ctx.kv_write(nk, nv, sl, kr, vr, 1, 16, blk)
+                ctx.attn_decode_sa_compact(qd, kr, vr, sl, outs[3], 1 / math.sqrt(d), 1, 16, blk)
 
         # The caches are state (appends; the ring reuses slots), so every run starts from
         # the same contents.
@@ -67,7 +76,7 @@ def test_routed_step_graph_replay_matches_eager():
             sl.fill_(s_val)
             step()
             ctx.check()
-            results[s_val] = [o.clone() for o in outs]
+            results[s_val] = [o.clone() for o in outs] + [x.clone() for x in (kc, vc, kr, vr)]
 
         g = torch.cuda.CUDAGraph()
         cs = torch.cuda.Stream(dev)
@@ -83,6 +92,6 @@ def test_routed_step_graph_replay_matches_eager():
             g.replay()
             torch.cuda.synchronize()
             ctx.check()
-            for got, want in zip(outs, results[s_val]):
+            for got, want in zip(outs + [kc, vc, kr, vr], results[s_val]):
                 assert torch.equal(got, want), s_val
         del g
