@@ -745,7 +745,11 @@ def run_flux(args, rank, world, dev_index):
     h2d_bytes, d2h_bytes, launches = wl.h2d_bytes, wl.d2h_bytes, wl.launches * args.steps
     fa_avg = statistics.mean(fa_ms)
     sa_avg = statistics.mean(sa_ms)
-    peak_t = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    # The timed region is short (about 20 steps of 9 ms) and runs at the maximum SM clock
+    # (sampled below), so the kernel is compared with cuBLAS's burst figure; the sustained
+    # figure (a seconds-long loop settled under the power cap, at about 1.3 GHz) is context.
+    peak_t = peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained"))
+    peak_sus = peaks.get("bf16_tflops_sustained", peak_t)
     fa_tflops = wl.flops_fa / (fa_avg * 1e-3) / 1e12
     sa_tflops = wl.flops_sa / (sa_avg * 1e-3) / 1e12
 
@@ -840,7 +844,8 @@ def run_flux(args, rank, world, dev_index):
                      "unit": "TFLOP/s", "frac": round(fa_tflops / peak_t, 4),
                      "traffic": recorded_traffic("prefill_fa_T32768"),
                      "kernel": "prefill_kernel<128> (FA layer)",
-                     "peak_source": f"{peak_src} bf16_tflops_sustained"},
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "frac_of_sustained": round(fa_tflops / peak_sus, 4)},
         "sa_prefill": {"TFLOP/s": round(sa_tflops, 1), "ms": round(sa_avg, 4),
                        "frac": round(sa_tflops / peak_t, 4)},
         "fa_prefill": {"TFLOP/s": round(fa_tflops, 1), "ms": round(fa_avg, 4)},
