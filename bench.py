@@ -252,6 +252,38 @@ class PrefillWorkload:
         for l in (0, 1):
             self.o_h[l].copy_(self.o[l], non_blocking=True)
 
+    def copy_floor_ms(self, reps=5):
+        """ms for one step's host<->device traffic alone: the inputs' upload and the two
+        outputs' download running concurrently on two streams (no compute) -- the floor
+        of the pipelined e2e step on this machine's PCIe link."""
+        import torch
+        s_in, s_out = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
+        src = (self.q_h, self.k_h, self.v_h, self.hidden_h)
+        dst = (self.q, self.k, self.v, self.hidden)
+
+        def once():
+            with torch.cuda.stream(s_in):
+                for d_, x in zip(dst, src):
+                    d_.copy_(x, non_blocking=True)
+            with torch.cuda.stream(s_out):
+                for l in (0, 1):
+                    self.o_h[l].copy_(self.o[l], non_blocking=True)
+        once()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            torch.cuda.current_stream().wait_stream(s_in)
+            torch.cuda.current_stream().wait_stream(s_out)
+            s_in.wait_stream(torch.cuda.current_stream())
+            s_out.wait_stream(torch.cuda.current_stream())
+            once()
+        torch.cuda.current_stream().wait_stream(s_in)
+        torch.cuda.current_stream().wait_stream(s_out)
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / reps
+
     def e2e_pipelined(self, steps):
         """The step from pinned host memory, pipelined over three streams: step k's compute
         overlaps step k+1's host->device copy of its inputs and step k-1's device->host copy
@@ -706,6 +738,7 @@ def run_flux(args, rank, world, dev_index):
     s1.synchronize()
     e2e_serial_ms = ranks_max(s0.elapsed_time(s1) / e2e_steps)
     e2e_serial_value = whole_job_rate(wl.flops, world, e2e_serial_ms)
+    copy_floor = wl.copy_floor_ms()
 
     # router latency: the step's router, and the 36-layer router (hidden 65536 x 2560,
     # MLP 5120 -> 512 -> 36); CUDA events around 20 back-to-back calls.
@@ -864,6 +897,10 @@ def run_flux(args, rank, world, dev_index):
                        "fill and drain included)",
                 "steps": e2e_steps,
                 "serial_ms_per_step": round(e2e_serial_ms, 4),
+                "copy_floor_ms_per_step": round(copy_floor, 4),
+                "copy_floor_note": "the step's upload and download alone, concurrently on two "
+                                   "streams, on this machine; e2e ms / this = the pipeline's "
+                                   "overhead over the PCIe floor",
                 "serial_value": round(e2e_serial_value, 2)},
         "gpu_launches": launches,
         "clocks": clocks,
