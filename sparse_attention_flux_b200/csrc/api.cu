@@ -87,6 +87,119 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 flux::DevStatus status_of(const flux_ctx* c) { return flux::DevStatus{c->err, c->spin_ns}; }
 
+// ---- decode entry points: one argument set, one set of host checks, one launch path
+struct DecodeCall {
+  const char* name;
+  const uint16_t* q;
+  const uint16_t* k_cache;
+  const uint16_t* v_cache;
+  int rows;                      // cache rows per sequence: S_max, or the ring's
+  const int32_t* seqlens;
+  uint16_t* o;
+  float* lse;
+  int B, Hq, Hkv, d;
+  const uint8_t* layer_mode;
+  int layer;
+  const uint8_t* head_mode;      // per-query-head routing, or null
+  int sink_blocks, window_blocks, block;
+  float scale;
+  int compact;                   // the cache is an SA ring of (sink + W) * block rows
+  const uint16_t* k_new;         // fused append of token seqlens[b] - 1, or null
+  const uint16_t* v_new;
+};
+
+// The checks every decode entry point shares; nothing is launched on failure.
+int check_decode(const DecodeCall& a, long long max_groups) {
+  if (!a.q || !a.k_cache || !a.v_cache || !a.seqlens || !a.o)
+    return fail(FLUX_ERR_INVALID_ARG, "%s: null tensor", a.name);
+  if (a.B < 1 || a.Hq < 1 || a.Hkv < 1 || a.rows < 1)
+    return fail(FLUX_ERR_SHAPE, "%s: sizes must be positive", a.name);
+  if (a.d != 64 && a.d != 128)
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: head_dim %d (supported: 64, 128)", a.name, a.d);
+  if (a.Hq % a.Hkv != 0 || (a.Hq / a.Hkv != 1 && a.Hq / a.Hkv != 2 && a.Hq / a.Hkv != 4))
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: Hq/Hkv must be 1, 2 or 4 (%d, %d)", a.name, a.Hq,
+                a.Hkv);
+  if (a.block < 1 || a.sink_blocks < 0 || a.window_blocks < 1)
+    return fail(FLUX_ERR_INVALID_ARG, "%s: bad block / sink / window", a.name);
+  if (a.compact && (a.block < 64 || a.block % 64 != 0))
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: a ring needs block a multiple of 64", a.name);
+  if (a.compact && static_cast<long long>(a.sink_blocks + a.window_blocks) * a.block != a.rows)
+    return fail(FLUX_ERR_SHAPE, "%s: ring rows must be (sink + window) * block", a.name);
+  if (a.layer_mode && a.layer < 0) return fail(FLUX_ERR_INVALID_ARG, "%s: negative layer", a.name);
+  if (!(a.scale == a.scale) || a.scale <= 0.f || a.scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "%s: scale must be finite and positive", a.name);
+  if (static_cast<long long>(a.B) * a.Hkv > max_groups)
+    return fail(FLUX_ERR_SHAPE, "%s: B * Hkv = %lld exceeds %lld", a.name,
+                static_cast<long long>(a.B) * a.Hkv, max_groups);
+  if (!aligned16(a.q) || !aligned16(a.k_cache) || !aligned16(a.v_cache) ||
+      (a.k_new && !aligned16(a.k_new)) || (a.v_new && !aligned16(a.v_new)))
+    return fail(FLUX_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", a.name);
+  return FLUX_OK;
+}
+
+// The call's split plan (a ring needs only its SA splits) and the bytes of its
+// split partials: o [B, Hq, nsplit, d] then (m, l), each 256-byte aligned.
+size_t plan_decode(const DecodeCall& a, int num_sms, flux::DecodeLaunch* p, size_t* o_bytes) {
+  flux::decode_plan(a.B, a.Hkv, a.rows, a.sink_blocks, a.window_blocks, a.block, num_sms,
+                    &p->nsplit, &p->chunk_fa, &p->tiles_sa);
+  if (a.compact)
+    p->nsplit = flux::decode_sa_splits(a.sink_blocks, a.window_blocks, a.block, p->tiles_sa);
+  const size_t rows = static_cast<size_t>(a.B) * a.Hq * p->nsplit;
+  *o_bytes = align256(rows * a.d * sizeof(float));
+  return *o_bytes + align256(rows * 2 * sizeof(float));
+}
+
+// Tensor maps and the launch, with the partials at `part`, the merge tickets
+// and the error word / wait bound given.
+int launch_decode_call(const DecodeCall& a, flux::DecodeLaunch& p, void* part, size_t o_bytes,
+                       int* tickets, flux::DevStatus st, cudaStream_t stream) {
+  CUtensorMap tk, tv;
+  int rc;
+  if ((rc = make_map_4d(&tk, a.k_cache, a.d, a.Hkv, a.rows, a.B, 64, 64)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, a.v_cache, a.d, a.Hkv, a.rows, a.B, 64, 64)) != FLUX_OK) return rc;
+  p.B = a.B;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.d = a.d;
+  p.S_max = a.rows;
+  p.q = a.q;
+  p.seqlens = a.seqlens;
+  p.o = a.o;
+  p.lse = a.lse;
+  p.layer_mode = a.layer_mode;
+  p.layer = a.layer;
+  p.sink_blocks = a.sink_blocks;
+  p.window_blocks = a.window_blocks;
+  p.block = a.block;
+  p.scale = a.scale;
+  p.compact = a.compact;
+  p.head_mode = a.head_mode;
+  p.part_o = static_cast<float*>(part);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(part) + o_bytes);
+  p.tickets = tickets;
+  p.st = st;
+  p.k_new = a.k_new;
+  p.v_new = a.v_new;
+  p.k_cache = const_cast<uint16_t*>(a.k_cache);
+  p.v_cache = const_cast<uint16_t*>(a.v_cache);
+  const cudaError_t e = flux::launch_decode(tk, tv, p, stream);
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, a.name);
+}
+
+// A decode call on a context: its workspace holds the partials.
+int run_decode(flux_ctx* c, const DecodeCall& a, flux_stream_t stream) {
+  if (!c) return fail(FLUX_ERR_INVALID_ARG, "%s: null context", a.name);
+  int rc = check_decode(a, kMaxTickets);
+  if (rc != FLUX_OK) return rc;
+  flux::DecodeLaunch p;
+  size_t o_bytes = 0;
+  const size_t need = plan_decode(a, c->num_sms, &p, &o_bytes);
+  if (need > c->workspace_bytes)
+    return fail(FLUX_ERR_SHAPE, "%s: workspace %zu < %zu bytes", a.name, c->workspace_bytes, need);
+  return launch_decode_call(a, p, c->workspace, o_bytes, c->tickets, status_of(c),
+                            static_cast<cudaStream_t>(stream));
+}
+
 }  // namespace
 
 extern "C" {
@@ -358,60 +471,10 @@ int flux_attn_decode(flux_ctx* c, const uint16_t* q, const uint16_t* k_cache,
                      float* lse, int B, int Hq, int Hkv, int d, const uint8_t* layer_mode,
                      int layer, int sink_blocks, int window_blocks, int block, float scale,
                      flux_stream_t stream) {
-  if (!c || !q || !k_cache || !v_cache || !seqlens || !o)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: null tensor");
-  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode: sizes must be positive");
-  if (d != 64 && d != 128)
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode: head_dim %d (supported: 64, 128)", d);
-  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode: Hq/Hkv must be 1, 2 or 4 (%d, %d)", Hq,
-                Hkv);
-  if (block < 1 || sink_blocks < 0 || window_blocks < 1)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: bad block / sink / window");
-  if (layer_mode && layer < 0) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: negative layer");
-  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: scale must be finite and positive");
-  if (static_cast<long long>(B) * Hkv > kMaxTickets)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode: B * Hkv > %d", kMaxTickets);
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode: tensors must be 16-byte aligned");
-  flux::DecodeLaunch p;
-  flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
-                    &p.chunk_fa, &p.tiles_sa);
-  const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
-  const size_t o_bytes = align256(rows * d * sizeof(float));
-  const size_t need = o_bytes + align256(rows * 2 * sizeof(float));
-  if (need > c->workspace_bytes)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode: workspace %zu < %zu bytes", c->workspace_bytes,
-                need);
-  CUtensorMap tk, tv;
-  int rc;
-  if ((rc = make_map_4d(&tk, k_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tv, v_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.d = d;
-  p.S_max = S_max;
-  p.q = q;
-  p.seqlens = seqlens;
-  p.o = o;
-  p.lse = lse;
-  p.layer_mode = layer_mode;
-  p.layer = layer;
-  p.sink_blocks = sink_blocks;
-  p.window_blocks = window_blocks;
-  p.block = block;
-  p.scale = scale;
-  p.part_o = static_cast<float*>(c->workspace);
-  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
-  p.tickets = c->tickets;
-  p.compact = 0;
-  p.head_mode = nullptr;
-  p.st = status_of(c);
-  const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode: launch");
+  const DecodeCall a{"flux_attn_decode", q, k_cache, v_cache, S_max, seqlens, o, lse, B, Hq, Hkv,
+                     d, layer_mode, layer, nullptr, sink_blocks, window_blocks, block, scale,
+                     0, nullptr, nullptr};
+  return run_decode(c, a, stream);
 }
 
 int flux_kv_write(flux_ctx* c, const uint16_t* k_src, const uint16_t* v_src, int n_src,
@@ -439,58 +502,13 @@ int flux_attn_decode_sa_compact(flux_ctx* c, const uint16_t* q, const uint16_t* 
                                 const uint16_t* v_ring, const int32_t* seqlens, uint16_t* o,
                                 float* lse, int B, int Hq, int Hkv, int d, int sink_blocks,
                                 int window_blocks, int block, float scale, flux_stream_t stream) {
-  if (!c || !q || !k_ring || !v_ring || !seqlens || !o)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: null tensor");
-  if (B < 1 || Hq < 1 || Hkv < 1 || sink_blocks < 0 || window_blocks < 1)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: bad sizes");
-  if (d != 64 && d != 128)
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_sa_compact: head_dim %d", d);
-  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_sa_compact: Hq/Hkv must be 1, 2 or 4");
-  if (block < 64 || block % 64 != 0)
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_sa_compact: block must be a multiple of 64");
-  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: scale must be finite and positive");
-  if (static_cast<long long>(B) * Hkv > kMaxTickets)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_sa_compact: B * Hkv > %d", kMaxTickets);
-  if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring))
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: tensors must be 16-byte aligned");
-  const int rows = (sink_blocks + window_blocks) * block;
-  flux::DecodeLaunch p;
-  flux::decode_plan(B, Hkv, rows, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
-                    &p.chunk_fa, &p.tiles_sa);
-  p.nsplit = flux::decode_sa_splits(sink_blocks, window_blocks, block, p.tiles_sa);  // SA only
-  const size_t nrow = static_cast<size_t>(B) * Hq * p.nsplit;
-  const size_t o_bytes = align256(nrow * d * sizeof(float));
-  if (o_bytes + align256(nrow * 2 * sizeof(float)) > c->workspace_bytes)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_sa_compact: workspace too small");
-  CUtensorMap tk, tv;
-  int rc;
-  if ((rc = make_map_4d(&tk, k_ring, d, Hkv, rows, B, 64, 64)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tv, v_ring, d, Hkv, rows, B, 64, 64)) != FLUX_OK) return rc;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.d = d;
-  p.S_max = rows;
-  p.q = q;
-  p.seqlens = seqlens;
-  p.o = o;
-  p.lse = lse;
-  p.layer_mode = nullptr;
-  p.layer = 0;
-  p.sink_blocks = sink_blocks;
-  p.window_blocks = window_blocks;
-  p.block = block;
-  p.scale = scale;
-  p.part_o = static_cast<float*>(c->workspace);
-  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
-  p.tickets = c->tickets;
-  p.compact = 1;
-  p.head_mode = nullptr;
-  p.st = status_of(c);
-  const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_sa_compact: launch");
+  const long long rows = static_cast<long long>(sink_blocks + window_blocks) * block;
+  if (rows < 1 || rows > (1LL << 30))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_sa_compact: bad sink / window / block");
+  const DecodeCall a{"flux_attn_decode_sa_compact", q, k_ring, v_ring, static_cast<int>(rows),
+                     seqlens, o, lse, B, Hq, Hkv, d, nullptr, 0, nullptr, sink_blocks,
+                     window_blocks, block, scale, 1, nullptr, nullptr};
+  return run_decode(c, a, stream);
 }
 
 int flux_attn_decode_append(flux_ctx* c, const uint16_t* q, const uint16_t* k_new,
@@ -499,70 +517,14 @@ int flux_attn_decode_append(flux_ctx* c, const uint16_t* q, const uint16_t* k_ne
                             int B, int Hq, int Hkv, int d, const uint8_t* layer_mode, int layer,
                             int sink_blocks, int window_blocks, int block, int compact,
                             float scale, flux_stream_t stream) {
-  static const char* name = "flux_attn_decode_append";
-  if (!c || !q || !k_new || !v_new || !k_cache || !v_cache || !seqlens || !o)
-    return fail(FLUX_ERR_INVALID_ARG, "%s: null tensor", name);
-  if (B < 1 || Hq < 1 || Hkv < 1 || cache_rows < 1)
-    return fail(FLUX_ERR_SHAPE, "%s: sizes must be positive", name);
-  if (d != 64 && d != 128)
-    return fail(FLUX_ERR_UNSUPPORTED, "%s: head_dim %d (supported: 64, 128)", name, d);
-  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
-    return fail(FLUX_ERR_UNSUPPORTED, "%s: Hq/Hkv must be 1, 2 or 4 (%d, %d)", name, Hq, Hkv);
-  if (block < 1 || sink_blocks < 0 || window_blocks < 1 || (compact != 0 && compact != 1))
-    return fail(FLUX_ERR_INVALID_ARG, "%s: bad block / sink / window / compact", name);
-  if (compact && (block < 64 || block % 64 != 0))
-    return fail(FLUX_ERR_UNSUPPORTED, "%s: a ring needs block a multiple of 64", name);
-  if (compact && static_cast<long long>(sink_blocks + window_blocks) * block != cache_rows)
-    return fail(FLUX_ERR_SHAPE, "%s: ring cache_rows must be (sink + window) * block", name);
-  if (!compact && layer_mode && layer < 0)
-    return fail(FLUX_ERR_INVALID_ARG, "%s: negative layer", name);
-  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
-    return fail(FLUX_ERR_INVALID_ARG, "%s: scale must be finite and positive", name);
-  if (static_cast<long long>(B) * Hkv > kMaxTickets)
-    return fail(FLUX_ERR_SHAPE, "%s: B * Hkv > %d", name, kMaxTickets);
-  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
-      !aligned16(v_cache))
-    return fail(FLUX_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", name);
-  flux::DecodeLaunch p;
-  flux::decode_plan(B, Hkv, cache_rows, sink_blocks, window_blocks, block, c->num_sms,
-                    &p.nsplit, &p.chunk_fa, &p.tiles_sa);
-  if (compact) p.nsplit = flux::decode_sa_splits(sink_blocks, window_blocks, block, p.tiles_sa);
-  const size_t nrow = static_cast<size_t>(B) * Hq * p.nsplit;
-  const size_t o_bytes = align256(nrow * d * sizeof(float));
-  const size_t need = o_bytes + align256(nrow * 2 * sizeof(float));
-  if (need > c->workspace_bytes)
-    return fail(FLUX_ERR_SHAPE, "%s: workspace %zu < %zu bytes", name, c->workspace_bytes, need);
-  CUtensorMap tk, tv;
-  int rc;
-  if ((rc = make_map_4d(&tk, k_cache, d, Hkv, cache_rows, B, 64, 64)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tv, v_cache, d, Hkv, cache_rows, B, 64, 64)) != FLUX_OK) return rc;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.d = d;
-  p.S_max = cache_rows;
-  p.q = q;
-  p.seqlens = seqlens;
-  p.o = o;
-  p.lse = lse;
-  p.layer_mode = compact ? nullptr : layer_mode;
-  p.layer = compact ? 0 : layer;
-  p.sink_blocks = sink_blocks;
-  p.window_blocks = window_blocks;
-  p.block = block;
-  p.scale = scale;
-  p.part_o = static_cast<float*>(c->workspace);
-  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
-  p.tickets = c->tickets;
-  p.compact = compact;
-  p.head_mode = nullptr;
-  p.st = status_of(c);
-  p.k_new = k_new;
-  p.v_new = v_new;
-  p.k_cache = k_cache;
-  p.v_cache = v_cache;
-  const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_append: launch");
+  if (!k_new || !v_new)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_append: null k_new / v_new");
+  if (compact != 0 && compact != 1)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_append: compact must be 0 or 1");
+  const DecodeCall a{"flux_attn_decode_append", q, k_cache, v_cache, cache_rows, seqlens, o, lse,
+                     B, Hq, Hkv, d, compact ? nullptr : layer_mode, compact ? 0 : layer, nullptr,
+                     sink_blocks, window_blocks, block, scale, compact, k_new, v_new};
+  return run_decode(c, a, stream);
 }
 
 }  // extern "C"
@@ -626,43 +588,21 @@ extern "C" int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cac
                                         int Hq, int Hkv, int d, const uint8_t* layer_mode,
                                         int layer, int sink_blocks, int window_blocks, int block,
                                         float scale, int32_t* status, flux_stream_t stream) {
-  if (!q || !k_cache || !v_cache || !seqlens || !o)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: null tensor");
-  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_noalloc: sizes must be positive");
-  if (d != 64 && d != 128)
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_noalloc: head_dim %d (supported: 64, 128)",
-                d);
-  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_noalloc: Hq/Hkv must be 1, 2 or 4");
-  if (block < 1 || sink_blocks < 0 || window_blocks < 1)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: bad block / sink / window");
-  if (layer_mode && layer < 0)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: negative layer");
-  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: scale must be finite and positive");
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_noalloc: tensors must be 16-byte aligned");
-  if (static_cast<long long>(B) * Hkv > kNoAllocMaxGroups)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_noalloc: B * Hkv = %lld exceeds %d",
-                static_cast<long long>(B) * Hkv, kNoAllocMaxGroups);
-  NoAllocDevice* dev = nullptr;
-  int rc = noalloc_setup(&dev);
+  const DecodeCall a{"flux_attn_decode_noalloc", q, k_cache, v_cache, S_max, seqlens, o, lse, B,
+                     Hq, Hkv, d, layer_mode, layer, nullptr, sink_blocks, window_blocks, block,
+                     scale, 0, nullptr, nullptr};
+  int rc = check_decode(a, kNoAllocMaxGroups);
   if (rc != FLUX_OK) return rc;
+  NoAllocDevice* dev = nullptr;
+  if ((rc = noalloc_setup(&dev)) != FLUX_OK) return rc;
   flux::DecodeLaunch p;
-  flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, dev->num_sms, &p.nsplit,
-                    &p.chunk_fa, &p.tiles_sa);
-  const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
-  const size_t ml_bytes = align256(rows * 2 * sizeof(float));
-  const size_t o_bytes = align256(rows * d * sizeof(float));
-  if (kNoAllocPartOff + ml_bytes + o_bytes > kNoAllocBytes)
+  size_t o_bytes = 0;
+  const size_t need = plan_decode(a, dev->num_sms, &p, &o_bytes);
+  if (kNoAllocPartOff + need > kNoAllocBytes)
     return fail(FLUX_ERR_SHAPE,
                 "flux_attn_decode_noalloc: %zu bytes of split partials exceed the %zu-byte static "
                 "scratch (use flux_attn_decode with a ctx for this shape)",
-                ml_bytes + o_bytes, kNoAllocBytes - kNoAllocPartOff);
-  CUtensorMap tk, tv;
-  if ((rc = make_map_4d(&tk, k_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tv, v_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
+                need, kNoAllocBytes - kNoAllocPartOff);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* err = reinterpret_cast<int*>(dev->base + kNoAllocErrOff);
   int* tickets = reinterpret_cast<int*>(dev->base + kNoAllocTicketOff);
@@ -672,29 +612,9 @@ extern "C" int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cac
   if (e == cudaSuccess)
     e = cudaMemsetAsync(tickets, 0, static_cast<size_t>(B) * Hkv * sizeof(int), s);
   if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: clear scratch");
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.d = d;
-  p.S_max = S_max;
-  p.q = q;
-  p.seqlens = seqlens;
-  p.o = o;
-  p.lse = lse;
-  p.layer_mode = layer_mode;
-  p.layer = layer;
-  p.sink_blocks = sink_blocks;
-  p.window_blocks = window_blocks;
-  p.block = block;
-  p.scale = scale;
-  p.part_ml = reinterpret_cast<float*>(dev->base + kNoAllocPartOff);
-  p.part_o = reinterpret_cast<float*>(dev->base + kNoAllocPartOff + ml_bytes);
-  p.tickets = tickets;
-  p.compact = 0;
-  p.head_mode = nullptr;
-  p.st = flux::DevStatus{err, 2000LL * 1000000LL};
-  e = flux::launch_decode(tk, tv, p, s);
-  if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: launch");
+  rc = launch_decode_call(a, p, dev->base + kNoAllocPartOff, o_bytes, tickets,
+                          flux::DevStatus{err, 2000LL * 1000000LL}, s);
+  if (rc != FLUX_OK) return rc;
   if (status && (e = cudaMemcpyAsync(status, err, sizeof(int), cudaMemcpyDeviceToDevice, s)) !=
                     cudaSuccess)
     return cuda_fail(e, "flux_attn_decode_noalloc: copy status");
@@ -763,55 +683,10 @@ extern "C" int flux_attn_decode_heads(flux_ctx* c, const uint16_t* q, const uint
                                       const uint8_t* head_mode, int sink_blocks, int window_blocks,
                                       int block, float scale, flux_stream_t stream) {
   if (!head_mode) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: head_mode is required");
-  if (!c || !q || !k_cache || !v_cache || !seqlens || !o)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: null tensor");
-  if (B < 1 || Hq < 1 || Hkv < 1 || S_max < 1)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_heads: sizes must be positive");
-  if (d != 64 && d != 128) return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_heads: head_dim %d", d);
-  if (Hq % Hkv != 0 || (Hq / Hkv != 1 && Hq / Hkv != 2 && Hq / Hkv != 4))
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_heads: Hq/Hkv must be 1, 2 or 4");
-  if (block < 1 || sink_blocks < 0 || window_blocks < 1)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: bad block / sink / window");
-  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: scale must be finite and positive");
-  if (static_cast<long long>(B) * Hkv > kMaxTickets)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_heads: B * Hkv > %d", kMaxTickets);
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_decode_heads: tensors must be 16-byte aligned");
-  flux::DecodeLaunch p;
-  flux::decode_plan(B, Hkv, S_max, sink_blocks, window_blocks, block, c->num_sms, &p.nsplit,
-                    &p.chunk_fa, &p.tiles_sa);
-  const size_t rows = static_cast<size_t>(B) * Hq * p.nsplit;
-  const size_t o_bytes = align256(rows * d * sizeof(float));
-  if (o_bytes + align256(rows * 2 * sizeof(float)) > c->workspace_bytes)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_decode_heads: workspace too small");
-  CUtensorMap tk, tv;
-  int rc;
-  if ((rc = make_map_4d(&tk, k_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tv, v_cache, d, Hkv, S_max, B, 64, 64)) != FLUX_OK) return rc;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.d = d;
-  p.S_max = S_max;
-  p.q = q;
-  p.seqlens = seqlens;
-  p.o = o;
-  p.lse = lse;
-  p.layer_mode = nullptr;
-  p.layer = 0;
-  p.sink_blocks = sink_blocks;
-  p.window_blocks = window_blocks;
-  p.block = block;
-  p.scale = scale;
-  p.part_o = static_cast<float*>(c->workspace);
-  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(c->workspace) + o_bytes);
-  p.tickets = c->tickets;
-  p.compact = 0;
-  p.head_mode = head_mode;
-  p.st = status_of(c);
-  const cudaError_t e = flux::launch_decode(tk, tv, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_decode_heads: launch");
+  const DecodeCall a{"flux_attn_decode_heads", q, k_cache, v_cache, S_max, seqlens, o, lse, B, Hq,
+                     Hkv, d, nullptr, 0, head_mode, sink_blocks, window_blocks, block, scale, 0,
+                     nullptr, nullptr};
+  return run_decode(c, a, stream);
 }
 
 // ---------------------------------------------------------------------------

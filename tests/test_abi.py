@@ -57,3 +57,36 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(flux, "_lib", None)
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         flux.lib()
+
+
+def test_decode_family_host_checks_need_no_gpu(lib):
+    """The decode entry points share one set of host checks: each rejects a null context or
+    tensor, an unsupported group size, a ring of the wrong size, a bad scale or too many
+    (sequence, kv head) groups before any CUDA call."""
+    P = ctypes.c_void_p(256)                      # aligned, never dereferenced
+    ctx = ctypes.c_void_p(4096)                   # never dereferenced: checks fail first
+    # flux_attn_decode: null context
+    assert lib.flux_attn_decode(None, P, P, P, 64, P, P, None, 1, 2, 1, 64, None, 0, 1, 1, 64,
+                                0.1, None) == flux.FLUX_ERR_INVALID_ARG
+    assert b"null" in lib.flux_last_error()
+    # group size 3 is not supported
+    assert lib.flux_attn_decode(ctx, P, P, P, 64, P, P, None, 1, 3, 1, 64, None, 0, 1, 1, 64,
+                                0.1, None) == flux.FLUX_ERR_UNSUPPORTED
+    # non-finite scale
+    assert lib.flux_attn_decode_heads(ctx, P, P, P, 64, P, P, None, 1, 2, 1, 64, P, 1, 1, 64,
+                                      float("nan"), None) == flux.FLUX_ERR_INVALID_ARG
+    # fused append: ring rows must be (sink + window) * block
+    assert lib.flux_attn_decode_append(ctx, P, P, P, P, P, 100, P, P, None, 1, 2, 1, 64, None, 0,
+                                       1, 1, 64, 1, 0.1, None) == flux.FLUX_ERR_SHAPE
+    assert lib.flux_attn_decode_append(ctx, P, None, P, P, P, 128, P, P, None, 1, 2, 1, 64, None,
+                                       0, 1, 1, 64, 1, 0.1, None) == flux.FLUX_ERR_INVALID_ARG
+    # compact ring decode: block must be a multiple of 64
+    assert lib.flux_attn_decode_sa_compact(ctx, P, P, P, P, P, None, 1, 2, 1, 64, 1, 1, 96, 0.1,
+                                           None) == flux.FLUX_ERR_UNSUPPORTED
+    # no-allocation decode: at most 4096 (sequence, kv head) groups
+    assert lib.flux_attn_decode_noalloc(P, P, P, 64, P, P, None, 8192, 2, 1, 64, None, 0, 1, 1,
+                                        64, 0.1, None, None) == flux.FLUX_ERR_SHAPE
+    assert b"4096" in lib.flux_last_error()
+    # misaligned cache pointer
+    assert lib.flux_attn_decode(ctx, P, ctypes.c_void_p(258), P, 64, P, P, None, 1, 2, 1, 64,
+                                None, 0, 1, 1, 64, 0.1, None) == flux.FLUX_ERR_INVALID_ARG
