@@ -87,6 +87,92 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 flux::DevStatus status_of(const flux_ctx* c) { return flux::DevStatus{c->err, c->spin_ns}; }
 
+// ---- prefill entry points: one argument set, one set of host checks, one launch path
+struct PrefillCall {
+  const char* name;
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  uint16_t* o;
+  float* lse;
+  int B, T, Hq, Hkv, d;
+  const uint8_t* layer_mode;
+  int layer;
+  const int32_t* row_ptr;
+  const int32_t* col;
+  int nqb, block;
+  float scale;
+  int force_mode;                // -1: layer_mode / head_mode decide; 0: SA; 1: FA
+  const uint8_t* head_mode;      // per-query-head routing, or null
+  const float* blend_score;      // soft routing: blend into o with r = score[layer], or null
+};
+
+// The checks every prefill entry point shares; nothing is launched on failure.
+// A call that may take the SA path needs the CSR block index.
+int check_prefill(const PrefillCall& a) {
+  if (!a.q || !a.k || !a.v || !a.o) return fail(FLUX_ERR_INVALID_ARG, "%s: null tensor", a.name);
+  if (a.B < 1 || a.T < 1 || a.Hq < 1 || a.Hkv < 1)
+    return fail(FLUX_ERR_SHAPE, "%s: sizes must be positive", a.name);
+  if (a.d != 64 && a.d != 128)
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: head_dim %d (supported: 64, 128)", a.name, a.d);
+  if (a.Hq % a.Hkv != 0)
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: Hq %% Hkv != 0 (%d, %d)", a.name, a.Hq, a.Hkv);
+  if (a.block != 64 && (a.block < 128 || a.block % 128 != 0))
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: block %d (64 or a multiple of 128)", a.name, a.block);
+  if (!(a.scale == a.scale) || a.scale <= 0.f || a.scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "%s: scale must be finite and positive", a.name);
+  if ((a.layer_mode || a.blend_score) && a.layer < 0)
+    return fail(FLUX_ERR_INVALID_ARG, "%s: negative layer", a.name);
+  const bool routed = a.layer_mode || a.head_mode || a.force_mode == 0;
+  if (routed) {
+    if (!a.row_ptr || !a.col)
+      return fail(FLUX_ERR_INVALID_ARG, "%s: row_ptr/col are required for a routed call", a.name);
+    if (a.nqb < (a.T + a.block - 1) / a.block)
+      return fail(FLUX_ERR_SHAPE, "%s: nqb %d < ceil(T / block) = %d", a.name, a.nqb,
+                  (a.T + a.block - 1) / a.block);
+    if ((a.T + 127) / 128 > flux::kPrefillMaxKvTiles)
+      return fail(FLUX_ERR_SHAPE, "%s: routed prefill supports T <= %d", a.name,
+                  flux::kPrefillMaxKvTiles * 128);
+  }
+  if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.o))
+    return fail(FLUX_ERR_INVALID_ARG, "%s: tensors must be 16-byte aligned", a.name);
+  return FLUX_OK;
+}
+
+// Checks, tensor maps and the launch of one prefill pass on a context.
+int run_prefill(flux_ctx* c, const PrefillCall& a, flux_stream_t stream) {
+  if (!c) return fail(FLUX_ERR_INVALID_ARG, "%s: null context", a.name);
+  int rc = check_prefill(a);
+  if (rc != FLUX_OK) return rc;
+  CUtensorMap tq, tk, tv, to;
+  if ((rc = make_map_4d(&tq, a.q, a.d, a.Hq, a.T, a.B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tk, a.k, a.d, a.Hkv, a.T, a.B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tv, a.v, a.d, a.Hkv, a.T, a.B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&to, a.o, a.d, a.Hq, a.T, a.B, 64, 128)) != FLUX_OK) return rc;
+  const bool routed = a.layer_mode || a.head_mode || a.force_mode == 0;
+  flux::PrefillLaunch p;
+  p.B = a.B;
+  p.T = a.T;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.d = a.d;
+  p.block = a.block;
+  p.nqb = routed ? a.nqb : 0;
+  p.scale = a.scale;
+  p.layer_mode = a.layer_mode;
+  p.layer = a.layer;
+  p.row_ptr = a.row_ptr;
+  p.col = a.col;
+  p.o = a.o;
+  p.lse = a.lse;
+  p.force_mode = a.force_mode;
+  p.head_mode = a.head_mode;
+  p.blend_score = a.blend_score;
+  p.st = status_of(c);
+  const cudaError_t e = flux::launch_prefill(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, a.name);
+}
+
 // ---- decode entry points: one argument set, one set of host checks, one launch path
 struct DecodeCall {
   const char* name;
@@ -356,103 +442,26 @@ int flux_attn_prefill(flux_ctx* c, const uint16_t* q, const uint16_t* k, const u
                       const uint8_t* layer_mode, int layer, const int32_t* row_ptr,
                       const int32_t* col, int nqb, int block, float scale,
                       flux_stream_t stream) {
-  if (!c || !q || !k || !v || !o) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: null tensor");
-  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill: sizes must be positive");
-  if (d != 64 && d != 128)
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill: head_dim %d (supported: 64, 128)", d);
-  if (Hq % Hkv != 0)
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill: Hq %% Hkv != 0 (%d, %d)", Hq, Hkv);
-  if (block != 64 && (block < 128 || block % 128 != 0))
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill: block %d (64 or a multiple of 128)",
-                block);
-  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: scale must be finite and positive");
-  if (layer_mode) {
-    if (layer < 0) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: negative layer");
-    if (!row_ptr || !col)
-      return fail(FLUX_ERR_INVALID_ARG,
-                  "flux_attn_prefill: row_ptr/col are required when layer_mode is given");
-    if (nqb < (T + block - 1) / block)
-      return fail(FLUX_ERR_SHAPE, "flux_attn_prefill: nqb %d < ceil(T / block) = %d", nqb,
-                  (T + block - 1) / block);
-    if ((T + 127) / 128 > flux::kPrefillMaxKvTiles)
-      return fail(FLUX_ERR_SHAPE, "flux_attn_prefill: routed prefill supports T <= %d",
-                  flux::kPrefillMaxKvTiles * 128);
-  }
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill: tensors must be 16-byte aligned");
-  CUtensorMap tq, tk, tv, to;
-  int rc;
-  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&to, o, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
-  flux::PrefillLaunch p;
-  p.B = B;
-  p.T = T;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.d = d;
-  p.block = block;
-  p.nqb = layer_mode ? nqb : 0;
-  p.scale = scale;
-  p.layer_mode = layer_mode;
-  p.layer = layer;
-  p.row_ptr = row_ptr;
-  p.col = col;
-  p.o = o;
-  p.lse = lse;
-  p.force_mode = -1;
-  p.head_mode = nullptr;
-  p.blend_score = nullptr;
-  p.st = status_of(c);
-  const cudaError_t e = flux::launch_prefill(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill: launch");
+  const PrefillCall a{"flux_attn_prefill", q, k, v, o, lse, B, T, Hq, Hkv, d, layer_mode, layer,
+                      row_ptr, col, nqb, block, scale, -1, nullptr, nullptr};
+  return run_prefill(c, a, stream);
 }
 
 int flux_attn_prefill_soft(flux_ctx* c, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                            uint16_t* o, int B, int T, int Hq, int Hkv, int d, const float* score,
                            int layer, const int32_t* row_ptr, const int32_t* col, int nqb,
                            int block, float scale, flux_stream_t stream) {
-  if (!score || layer < 0)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_soft: score and a layer are required");
-  if (!row_ptr || !col)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_soft: row_ptr/col are required");
-  if (block > 0 && T > 0 && nqb < (T + block - 1) / block)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_soft: nqb %d < ceil(T / block)", nqb);
-  if (T > 0 && (T + 127) / 128 > flux::kPrefillMaxKvTiles)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_soft: T <= %d", flux::kPrefillMaxKvTiles * 128);
-  // Argument checks and tensor maps exactly as flux_attn_prefill (FA pass first).
-  int rc = flux_attn_prefill(c, q, k, v, o, nullptr, B, T, Hq, Hkv, d, nullptr, 0, row_ptr, col,
-                             nqb, block, scale, stream);
+  if (!score) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_soft: score is required");
+  // The SA pass is checked first, so that nothing is launched if either pass would fail.
+  const PrefillCall sa{"flux_attn_prefill_soft", q, k, v, o, nullptr, B, T, Hq, Hkv, d, nullptr,
+                       layer, row_ptr, col, nqb, block, scale, 0, nullptr, score};
+  int rc = check_prefill(sa);
   if (rc != FLUX_OK) return rc;
-  CUtensorMap tq, tk, tv, to;
-  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&to, o, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
-  flux::PrefillLaunch p;
-  p.B = B;
-  p.T = T;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.d = d;
-  p.block = block;
-  p.nqb = nqb;
-  p.scale = scale;
-  p.layer_mode = nullptr;
-  p.layer = layer;
-  p.row_ptr = row_ptr;
-  p.col = col;
-  p.o = o;
-  p.lse = nullptr;
-  p.force_mode = 0;          // the SA pass, blended into the FA output in its epilogue
-  p.head_mode = nullptr;
-  p.blend_score = score;
-  p.st = status_of(c);
-  const cudaError_t e = flux::launch_prefill(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill_soft: launch");
+  // FA pass into o, then the SA pass whose epilogue blends r * o_FA + (1 - r) * o_SA.
+  const PrefillCall fa{"flux_attn_prefill_soft", q, k, v, o, nullptr, B, T, Hq, Hkv, d, nullptr,
+                       layer, row_ptr, col, nqb, block, scale, 1, nullptr, nullptr};
+  if ((rc = run_prefill(c, fa, stream)) != FLUX_OK) return rc;
+  return run_prefill(c, sa, stream);
 }
 
 int flux_decode_workspace_bytes(flux_ctx* c, int B, int Hq, int Hkv, int d, int S_max,
@@ -630,51 +639,9 @@ extern "C" int flux_attn_prefill_heads(flux_ctx* c, const uint16_t* q, const uin
                                        const int32_t* row_ptr, const int32_t* col, int nqb,
                                        int block, float scale, flux_stream_t stream) {
   if (!head_mode) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: head_mode is required");
-  if (!row_ptr || !col)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: row_ptr/col are required");
-  if (block > 0 && T > 0 && nqb < (T + block - 1) / block)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_heads: nqb %d < ceil(T / block)", nqb);
-  if (T > 0 && (T + 127) / 128 > flux::kPrefillMaxKvTiles)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_heads: T <= %d", flux::kPrefillMaxKvTiles * 128);
-  // Same checks as flux_attn_prefill (run with layer_mode absent, then relaunched per head).
-  if (!c || !q || !k || !v || !o) return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: null tensor");
-  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1)
-    return fail(FLUX_ERR_SHAPE, "flux_attn_prefill_heads: sizes must be positive");
-  if (d != 64 && d != 128) return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill_heads: head_dim %d", d);
-  if (Hq % Hkv != 0) return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill_heads: Hq %% Hkv != 0");
-  if (block != 64 && (block < 128 || block % 128 != 0))
-    return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_prefill_heads: block %d", block);
-  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: scale must be finite and positive");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
-    return fail(FLUX_ERR_INVALID_ARG, "flux_attn_prefill_heads: tensors must be 16-byte aligned");
-  CUtensorMap tq, tk, tv, to;
-  int rc;
-  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tv, v, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&to, o, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
-  flux::PrefillLaunch p;
-  p.B = B;
-  p.T = T;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.d = d;
-  p.block = block;
-  p.nqb = nqb;
-  p.scale = scale;
-  p.layer_mode = nullptr;
-  p.layer = 0;
-  p.row_ptr = row_ptr;
-  p.col = col;
-  p.o = o;
-  p.lse = lse;
-  p.force_mode = -1;
-  p.head_mode = head_mode;
-  p.blend_score = nullptr;
-  p.st = status_of(c);
-  const cudaError_t e = flux::launch_prefill(tq, tk, tv, to, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_attn_prefill_heads: launch");
+  const PrefillCall a{"flux_attn_prefill_heads", q, k, v, o, lse, B, T, Hq, Hkv, d, nullptr, 0,
+                      row_ptr, col, nqb, block, scale, -1, head_mode, nullptr};
+  return run_prefill(c, a, stream);
 }
 
 extern "C" int flux_attn_decode_heads(flux_ctx* c, const uint16_t* q, const uint16_t* k_cache,
