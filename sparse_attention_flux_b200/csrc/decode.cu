@@ -22,7 +22,7 @@
 //     active CTA of each (sequence, kv head) -- found by an atomic ticket, no
 //     spin -- merges the partial (o, m, l) of every active split; splits past
 //     the active range (most of an SA layer's grid) exit at entry.
-// About 110 registers and 97 KB of shared memory: two CTAs per SM.
+// About 156 registers (d 128) and 97 KB of shared memory: two CTAs per SM.
 #include <algorithm>
 
 #include "common.cuh"
