@@ -33,7 +33,6 @@ a bounded sample of the same workload, as the reference arm.
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import math
 import os
@@ -86,8 +85,9 @@ def sa_decode_tokens(s, block, sink, W):
 
 def recorded_traffic(key):
     """DRAM bytes per launch (read + write) of a kernel from its ncu capture, recorded in
-    profiles/dram_traffic.json together with a SHA-256 of the sources it was built from;
-    None when there is no record or any of those sources has changed since the capture."""
+    profiles/dram_traffic.json together with a SHA-256 of the code it was built from
+    (comments and whitespace removed); None when there is no record or that code has
+    changed since the capture."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
@@ -95,11 +95,8 @@ def recorded_traffic(key):
         rec = json.load(f).get(key)
     if not rec:
         return None
-    h = hashlib.sha256()
-    for rel in rec["sources"]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
-    if h.hexdigest() != rec["sources_sha256"]:
+    from sparse_attention_flux_b200.record_traffic import sources_sha256
+    if sources_sha256(rec["sources"]) != rec["sources_sha256"]:
         return None
     return int(rec["bytes_per_launch"])
 

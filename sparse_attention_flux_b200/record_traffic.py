@@ -7,8 +7,9 @@ Reads dram__bytes_read.sum and dram__bytes_write.sum of the (single) launch in
 an ncu report (``ncu -i REPORT --page raw --csv``), multiplies their sum by S
 (for a capture made on a smaller case whose traffic grows in proportion, e.g.
 batch 4 standing in for batch 16: S = 4) and stores it under KEY in
-profiles/dram_traffic.json together with a SHA-256 of the listed source files.
-bench.py reports the figure only while those files are unchanged.
+profiles/dram_traffic.json together with a SHA-256 of the listed source files'
+code (comments and whitespace removed).  bench.py reports the figure only while
+that code is unchanged.
 """
 from __future__ import annotations
 
@@ -18,6 +19,7 @@ import hashlib
 import io
 import json
 import os
+import re
 import subprocess
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -38,11 +40,20 @@ def dram_bytes(report: str) -> tuple[int, int]:
     return got[0], got[1]
 
 
+def code_of(text: str) -> str:
+    """C++ source with comments and whitespace removed: edits to comments or layout do
+    not change what the kernel is.  (The hashed sources hold no "//" or "/*" inside
+    string literals.)"""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return re.sub(r"\s+", "", text)
+
+
 def sources_sha256(sources) -> str:
     h = hashlib.sha256()
     for rel in sources:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            h.update(code_of(f.read()).encode())
     return h.hexdigest()
 
 
