@@ -26,9 +26,12 @@
 //   warps 4-7   softmax of Q0, warps 8-11 softmax of Q1: one query row per
 //               thread (= one TMEM lane); online softmax in the log2 domain;
 //               P_i written back over S_i's columns as packed bf16 for the
-//               TMEM-A MMA; O_i rescaled only when the row max grows by more
-//               than 2^8 (exact: the final division uses the same max); the
-//               epilogue writes O_i / l.
+//               TMEM-A MMA.  After a row's first tile the exponentials use
+//               the running max without the tile's row max (any max is exact
+//               as long as the final division uses it); the tile's row sum
+//               bounds every P, and only a sum above 2^20 sends the warp to
+//               the row max, a lazy rescale of l and O (growth above 2^8) and
+//               a redo of the tile.  The epilogue writes O_i / l.
 // TMEM columns: S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [384,384+D).
 #include "common.cuh"
 #include "kernels.h"
@@ -42,6 +45,7 @@ constexpr int kBN = 128;                  // key columns per tile
 constexpr int kChunkBytes = 128 * 128;    // 128 rows x 64 bf16: one swizzle-128B box
 constexpr int kThreads = 384;
 constexpr float kRescaleLog2 = 8.f;       // lazy rescale threshold, log2 units
+constexpr float kRedoSum = 1048576.f;     // 2^20: a tile row sum above it is redone
 
 struct PrefillArgs {
   int B, T, Hq, Hkv, G;
@@ -414,52 +418,94 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[c][e]);
       }
       const uint32_t sub = (mask >> (qs * 2)) & 3u;
-      if (J * kBN + kBN - 1 > t_row || sub != 3u) {
+      const bool need_mask = J * kBN + kBN - 1 > t_row || sub != 3u;
+      if (need_mask) {
 #pragma unroll
         for (int c = 0; c < kBN; ++c)
           if (J * kBN + c > t_row || !((sub >> (c >> 6)) & 1u)) x[c] = -INFINITY;
       }
-      // Row max with 8 independent accumulators (a 127-deep chain otherwise).
-      float mx[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = x[e];
-#pragma unroll
-      for (int c = 8; c < kBN; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      const float m_tile = mt * a.scale_log2;
-      const bool grow = m_tile > m_run + kRescaleLog2;
-      float alpha = 1.f;
-      if (grow) {
-        alpha = ex2(m_run - m_tile);
-        l_run *= alpha;
-        m_run = m_tile;
-      }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      // P = 2^(x scale - m) is exact for any m as long as the final division
+      // (and the LSE) use the same m and nothing overflows, so after a row's
+      // first visible tile the exponentials are taken against the running max
+      // m_run without the tile's row max: the row sum, computed anyway, bounds
+      // every P of the tile.  Only if some lane's sum passes kRedoSum (or is
+      // not finite) -- its scores grew by more than about 20 in log2 units, as
+      // at a planted needle -- does the warp take the row max, rescale l and O
+      // lazily (growth above 2^8) and redo the tile.  P <= 2^20 per tile keeps
+      // l and O far from fp32 overflow over any T this kernel takes.
       float rs[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial row sums
+      // xv(i) reads score i; unrolled, every index is a compile-time constant.
+      auto exp_pass = [&](float m_use, auto&& xv) {
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(x[c * 32 + 2 * e], a.scale_log2, -m_use));
-          const float p1 = ex2(fmaf(x[c * 32 + 2 * e + 1], a.scale_log2, -m_use));
-          rs[e & 3] += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2(fmaf(xv(c * 32 + 2 * e), a.scale_log2, -m_use));
+            const float p1 = ex2(fmaf(xv(c * 32 + 2 * e + 1), a.scale_log2, -m_use));
+            rs[e & 3] += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);   // P_i over S_i's first 64 columns
         }
-        tmem_st16(tS + c * 16, pk);   // P_i over S_i's first 64 columns
+      };
+      bool redo = m_run == -INFINITY;
+      if (!__any_sync(0xffffffffu, redo)) {
+        exp_pass(m_run, [&](int i) { return x[i]; });
+        redo = !((rs[0] + rs[1]) + (rs[2] + rs[3]) <= kRedoSum);
       }
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_i is stable: S_i(j) completing implies PV_i(j-1) completed, and
-        // PV_i(j) waits for this warpgroup's arrival below.
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tO + c * 32, v);
+      if (__any_sync(0xffffffffu, redo)) {
+        // P overwrote columns 0-63 only: scores 64-127 are read back from TMEM,
+        // 0-63 are still in registers.
+        float xh[kBN / 2];
+        {
+          uint32_t v[2][32];
+          tmem_ld32(tS + 64, v[0]);
+          tmem_ld32(tS + 96, v[1]);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-          tmem_st32(tO + c * 32, v);
+          for (int e = 0; e < 32; ++e) {
+            xh[e] = __uint_as_float(v[0][e]);
+            xh[32 + e] = __uint_as_float(v[1][e]);
+          }
+          if (need_mask) {
+#pragma unroll
+            for (int c = kBN / 2; c < kBN; ++c)
+              if (J * kBN + c > t_row || !((sub >> (c >> 6)) & 1u)) xh[c - kBN / 2] = -INFINITY;
+          }
+        }
+        auto xr = [&](int i) { return i < kBN / 2 ? x[i] : xh[i - kBN / 2]; };
+        // Row max with 8 independent accumulators (a 127-deep chain otherwise).
+        float mx[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = xr(e);
+#pragma unroll
+        for (int c = 8; c < kBN; ++c) mx[c & 7] = fmaxf(mx[c & 7], xr(c));
+        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float m_tile = mt * a.scale_log2;
+        const bool grow = m_tile > m_run + kRescaleLog2;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = ex2(m_run - m_tile);
+          l_run *= alpha;
+          m_run = m_tile;
+        }
+        rs[0] = rs[1] = rs[2] = rs[3] = 0.f;
+        tmem_wait_st();   // the first pass's P stores land before these replace them
+        exp_pass(m_run == -INFINITY ? 0.f : m_run, xr);
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O_i is stable: S_i(j) completing implies PV_i(j-1) completed, and
+          // PV_i(j) waits for this warpgroup's arrival below.
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st32(tO + c * 32, v);
+          }
         }
       }
       l_run += (rs[0] + rs[1]) + (rs[2] + rs[3]);
