@@ -15,8 +15,9 @@
 //     of one query head, walking the union of the two tiles' lists.
 //
 // Per CTA (384 threads, warp-specialised):
-//   warp 0      TMA producer (Q0, Q1 once; K/V tiles into a 2-stage ring) and,
-//               for SA, the builder of the CTA's key-tile list.
+//   warp 0      TMA producer (Q0, Q1 once; K/V tiles into a 2-stage ring, K
+//               and V slots released separately) and, for SA, the builder of
+//               the CTA's key-tile list.
 //   warp 1      TMEM owner (all 512 columns) and UMMA issuer:
 //                 S_i = Q_i K^T             (A, B from shared memory)
 //                 O_i += P_i V              (A = P_i from TMEM, B from smem)
@@ -31,7 +32,8 @@
 //               as long as the final division uses it); the tile's row sum
 //               bounds every P, and only a sum above 2^20 sends the warp to
 //               the row max, a lazy rescale of l and O (growth above 2^8) and
-//               a redo of the tile.  The epilogue writes O_i / l.
+//               a redo of the tile.  The epilogue stages O_i / l as bf16 in
+//               Q_i's freed shared memory and stores it by TMA.
 // TMEM columns: S0 [0,128)  S1 [128,256)  O0 [256,256+D)  O1 [384,384+D).
 #include "common.cuh"
 #include "kernels.h"
