@@ -845,7 +845,7 @@ def run_flux(args, rank, world, dev_index):
         roof_dec = {"bound": "hbm", "achieved": round(fa_dec_gbs, 1), "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4),
                     "traffic": recorded_traffic("decode_fa_B16_S131072"),
-                    "kernel": "decode_kernel<128,4> (FA layer, incl. its append)"}
+                    "kernel": "decode_kernel<128> (FA layer, incl. its append)"}
         dec["roofline"] = roof_dec
         dec["routing_granularity"] = dw.granularity(8)
         dec["sa_layer"] = dw.sa_layer(10)

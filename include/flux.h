@@ -200,7 +200,8 @@ int flux_attn_prefill_soft(flux_ctx* ctx, const uint16_t* q, const uint16_t* k, 
  * all Hq/Hkv query heads of the group from that single read; the last CTA of
  * the group (atomic ticket, no spin) merges the partials.  Partials live in
  * the ctx workspace (flux_decode_workspace_bytes).  Supported: d 64/128,
- * Hq/Hkv in {1, 2, 4}.  Calls sharing a ctx must not overlap in time. */
+ * Hq/Hkv a whole number from 1 to 8 (else UNSUPPORTED).  Calls sharing a ctx
+ * must not overlap in time. */
 int flux_attn_decode(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_cache,
                      const uint16_t* v_cache, int S_max, const int32_t* seqlens,
                      uint16_t* o, float* lse, int B, int Hq, int Hkv, int d,

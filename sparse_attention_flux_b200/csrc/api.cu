@@ -202,9 +202,9 @@ int check_decode(const DecodeCall& a, long long max_groups) {
     return fail(FLUX_ERR_SHAPE, "%s: sizes must be positive", a.name);
   if (a.d != 64 && a.d != 128)
     return fail(FLUX_ERR_UNSUPPORTED, "%s: head_dim %d (supported: 64, 128)", a.name, a.d);
-  if (a.Hq % a.Hkv != 0 || (a.Hq / a.Hkv != 1 && a.Hq / a.Hkv != 2 && a.Hq / a.Hkv != 4))
-    return fail(FLUX_ERR_UNSUPPORTED, "%s: Hq/Hkv must be 1, 2 or 4 (%d, %d)", a.name, a.Hq,
-                a.Hkv);
+  if (a.Hq % a.Hkv != 0 || a.Hq / a.Hkv > flux::kDecodeMaxGroup)
+    return fail(FLUX_ERR_UNSUPPORTED, "%s: Hq/Hkv must be a whole number from 1 to %d (%d, %d)",
+                a.name, flux::kDecodeMaxGroup, a.Hq, a.Hkv);
   if (a.block < 1 || a.sink_blocks < 0 || a.window_blocks < 1)
     return fail(FLUX_ERR_INVALID_ARG, "%s: bad block / sink / window", a.name);
   if (a.compact && (a.block < 64 || a.block % 64 != 0))

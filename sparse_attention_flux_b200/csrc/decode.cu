@@ -15,14 +15,20 @@
 //     mbarrier that counts the four warps;
 //   * per warp, the group's scores S[G x 16] = Q K^T and values O += P V are
 //     16x8x16 warp MMAs (bf16 in, fp32 accumulate) fed by ldmatrix straight
-//     from the swizzled tiles -- the G query heads fill rows 0..G-1 of the
-//     16-row operand; online softmax in the log2 domain on the accumulator
-//     fragments, O rescaled only when a row max grows by more than 2^8;
+//     from the swizzled tiles -- the G <= 8 query heads fill rows 0..G-1 of the
+//     16-row operand (G is a launch argument, not a template parameter); online
+//     softmax in the log2 domain on the accumulator fragments, O rescaled only
+//     when a row max grows by more than 2^8;
 //   * the four warps' partials are merged in shared memory, then the last
 //     active CTA of each (sequence, kv head) -- found by an atomic ticket, no
 //     spin -- merges the partial (o, m, l) of every active split; splits past
-//     the active range (most of an SA layer's grid) exit at entry.
-// About 156 registers (d 128) and 97 KB of shared memory: two CTAs per SM.
+//     the active range (most of an SA layer's grid) exit at entry;
+//   * the cache is either full (row = position) or, for an SA layer, the
+//     compact ring of its sink blocks and last W blocks (block j >= sink in
+//     slot j mod W); with the step's new K/V rows passed in, the split that
+//     reads token s - 1 writes them into the cache before loading its tiles
+//     (the KV append fused into the decode launch).
+// About 160 registers (d 128) and 97 KB of shared memory: two CTAs per SM.
 #include <algorithm>
 
 #include "common.cuh"
@@ -37,6 +43,7 @@ constexpr int kStages = 3;
 constexpr int kComputeWarps = 4;
 constexpr int kThreads = 32 * (kComputeWarps + 1);
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kMaxGroup = kDecodeMaxGroup;   // query heads per kv head: operand rows 0..7
 
 template <int D>
 struct DSmem {
@@ -48,9 +55,10 @@ struct DSmem {
   static constexpr int FLAG = BARS + 2 * kStages * 8;
   static constexpr int TOTAL = FLAG + 16;
   static constexpr int ALLOC = TOTAL + 1024;
-  // After the stream: per-warp partials [warp][4 heads] m, l and o[warp][4][D].
-  static constexpr int CM = 0, CL = CM + kComputeWarps * 4 * 4, CO = CL + kComputeWarps * 4 * 4;
-  static_assert(CO + kComputeWarps * 4 * D * 4 <= BARS, "combine area must fit in the ring");
+  // After the stream: per-warp partials m, l [warp][kMaxGroup] and o[warp][kMaxGroup][D].
+  static constexpr int CM = 0, CL = CM + kComputeWarps * kMaxGroup * 4;
+  static constexpr int CO = CL + kComputeWarps * kMaxGroup * 4;
+  static_assert(CO + kComputeWarps * kMaxGroup * D * 4 <= BARS, "combine area must fit in the ring");
 };
 
 // A split's 64-token tiles.  FA: a contiguous token range.  SA: the sink
@@ -121,7 +129,7 @@ __device__ __forceinline__ Range split_range(const DecodeLaunch& a, bool fa, int
   return r;
 }
 
-template <int D, int G>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecodeLaunch a) {
@@ -140,13 +148,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   // leaves idle (launched for the FA range) only exit after them.
   const int i = blockIdx.z, g = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.Hq / a.Hkv;   // 1..kMaxGroup, checked on the host
   // Per-head routing: the group reads the FA range if any of its heads is FA;
   // its SA heads then mask every token outside the sink + window blocks.
   const uint8_t* hm = a.head_mode ? a.head_mode + g * G : nullptr;
   bool fa;
   if (hm) {
     fa = false;
-#pragma unroll
     for (int hh = 0; hh < G; ++hh) fa |= hm[hh] != 0;
   } else {
     fa = !a.compact && (a.layer_mode == nullptr || a.layer_mode[a.layer] != 0);
@@ -348,15 +356,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     float lq = l_part;
     lq += __shfl_xor_sync(0xffffffffu, lq, 1);
     lq += __shfl_xor_sync(0xffffffffu, lq, 2);
-    if (gq < 4) {
+    if (gq < G) {
       if (tq == 0) {
-        cm[warp * 4 + gq] = (ntiles > 0) ? m_run : -INFINITY;
-        cl[warp * 4 + gq] = (ntiles > 0) ? lq : 0.f;
+        cm[warp * kMaxGroup + gq] = (ntiles > 0) ? m_run : -INFINITY;
+        cl[warp * kMaxGroup + gq] = (ntiles > 0) ? lq : 0.f;
       }
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        co[(warp * 4 + gq) * D + 8 * n + 2 * tq] = oacc[n][0];
-        co[(warp * 4 + gq) * D + 8 * n + 2 * tq + 1] = oacc[n][1];
+        co[(warp * kMaxGroup + gq) * D + 8 * n + 2 * tq] = oacc[n][0];
+        co[(warp * kMaxGroup + gq) * D + 8 * n + 2 * tq + 1] = oacc[n][1];
       }
     }
   }
@@ -366,14 +374,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int hh = idx / D, c = idx % D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, cm[w * 4 + hh]);
+      for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, cm[w * kMaxGroup + hh]);
       float O = 0.f, Lsum = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
         for (int w = 0; w < kComputeWarps; ++w) {
-          const float wt = ex2(cm[w * 4 + hh] - M);
-          O += wt * co[(w * 4 + hh) * D + c];
-          Lsum += wt * cl[w * 4 + hh];
+          const float wt = ex2(cm[w * kMaxGroup + hh] - M);
+          O += wt * co[(w * kMaxGroup + hh) * D + c];
+          Lsum += wt * cl[w * kMaxGroup + hh];
         }
       }
       a.part_o[((grp + hh) * a.nsplit + i) * D + c] = O;
@@ -416,13 +424,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (tid == 0) a.tickets[b * a.Hkv + g] = 0;
 }
 
-template <int D, int G>
+template <int D>
 cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeLaunch& p,
                      cudaStream_t stream) {
   const int smem = DSmem<D>::ALLOC;
-  cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const dim3 grid(p.Hkv, p.B, p.nsplit);
-  decode_kernel<D, G><<<grid, kThreads, smem, stream>>>(tk, tv, p);
+  decode_kernel<D><<<grid, kThreads, smem, stream>>>(tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -485,15 +493,9 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int nsplit) {
 
 cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeLaunch& p,
                           cudaStream_t stream) {
-  const int G = p.Hq / p.Hkv;
-  if (p.d == 64) {
-    if (G == 1) return launch_t<64, 1>(tk, tv, p, stream);
-    if (G == 2) return launch_t<64, 2>(tk, tv, p, stream);
-    return launch_t<64, 4>(tk, tv, p, stream);
-  }
-  if (G == 1) return launch_t<128, 1>(tk, tv, p, stream);
-  if (G == 2) return launch_t<128, 2>(tk, tv, p, stream);
-  return launch_t<128, 4>(tk, tv, p, stream);
+  if (p.Hkv < 1 || p.Hq % p.Hkv != 0 || p.Hq / p.Hkv > kMaxGroup || (p.d != 64 && p.d != 128))
+    return cudaErrorInvalidValue;
+  return p.d == 64 ? launch_t<64>(tk, tv, p, stream) : launch_t<128>(tk, tv, p, stream);
 }
 
 }  // namespace flux

@@ -15,6 +15,10 @@ namespace flux {
 // at most this many 128-column key tiles, i.e. T <= 262144.
 constexpr int kPrefillMaxKvTiles = 2048;
 
+// Decode serves a kv head's whole query group from one read of its keys: the
+// group fills rows of a 16-row warp-MMA operand, at most this many query heads.
+constexpr int kDecodeMaxGroup = 8;
+
 struct PrefillLaunch {
   int B, T, Hq, Hkv, d;
   int block, nqb;

@@ -69,8 +69,11 @@ def test_decode_family_host_checks_need_no_gpu(lib):
     assert lib.flux_attn_decode(None, P, P, P, 64, P, P, None, 1, 2, 1, 64, None, 0, 1, 1, 64,
                                 0.1, None) == flux.FLUX_ERR_INVALID_ARG
     assert b"null" in lib.flux_last_error()
-    # group size 3 is not supported
-    assert lib.flux_attn_decode(ctx, P, P, P, 64, P, P, None, 1, 3, 1, 64, None, 0, 1, 1, 64,
+    # group sizes above 8 (and Hq not a multiple of Hkv) are not supported
+    assert lib.flux_attn_decode(ctx, P, P, P, 64, P, P, None, 1, 9, 1, 64, None, 0, 1, 1, 64,
+                                0.1, None) == flux.FLUX_ERR_UNSUPPORTED
+    assert b"1 to 8" in lib.flux_last_error()
+    assert lib.flux_attn_decode(ctx, P, P, P, 64, P, P, None, 1, 6, 4, 64, None, 0, 1, 1, 64,
                                 0.1, None) == flux.FLUX_ERR_UNSUPPORTED
     # non-finite scale
     assert lib.flux_attn_decode_heads(ctx, P, P, P, 64, P, P, None, 1, 2, 1, 64, P, 1, 1, 64,

@@ -41,6 +41,12 @@ CASES = [  # B, S_max, seqlens, Hq, Hkv, d, block, sink, W
     (1, 9000, [8999], 4, 4, 128, 128, 2, 4),
     (2, 777, [0, 776], 4, 2, 64, 64, 0, 1),
     (4, 2600, [2600, 2500, 130, 64], 32, 8, 128, 128, 1, 16),
+    # group sizes other than 1, 2, 4 (up to 8 query heads per kv head)
+    (2, 1500, [1500, 700], 6, 2, 128, 128, 1, 4),      # G 3
+    (1, 2100, [2033], 5, 1, 64, 64, 1, 5),            # G 5
+    (2, 1300, [1300, 1], 12, 2, 128, 64, 2, 3),       # G 6
+    (3, 900, [900, 450, 129], 7, 1, 64, 128, 0, 2),   # G 7
+    (2, 3000, [3000, 2999], 64, 8, 128, 128, 1, 16),  # G 8 (a 64 / 8 head layout)
 ]
 
 

@@ -77,3 +77,24 @@ def test_decode_per_head_matches_oracle(ctx, pattern):
                         window_blocks=W, block=block)
         ctx.check()
         assert torch.equal(o, o2)
+
+
+def test_decode_per_head_group_of_8(ctx):
+    # Eight query heads per kv head (the largest group decode takes), heads of one group
+    # routed differently: the group reads the FA range and its SA heads mask the rest.
+    B, S_max, Hq, Hkv, d, block, sink, W = 2, 3000, 16, 2, 128, 64, 1, 6
+    dev = ctx.device
+    q, kc, vc = synth.decode_inputs(B, S_max, Hq, Hkv, d, seed=78)
+    seqlens = np.array([3000, 1777], np.int32)
+    hm = (synth.rng(79).random(Hq) < 0.5).astype(np.uint8)
+    hm[:8] = [0, 1, 0, 0, 0, 0, 0, 0]          # group 0: one FA head among seven SA heads
+    qt, kt, vt = (synth.torch_from_bits(x).to(dev) for x in (q, kc, vc))
+    sl = torch.from_numpy(seqlens).to(dev)
+    o = torch.full_like(qt, float("nan"))
+    scale = 1 / math.sqrt(d)
+    ctx.attn_decode_heads(qt, kt, vt, sl, o, scale, torch.from_numpy(hm).to(dev), sink, W, block)
+    ctx.check()
+    fa, _ = oracle.attn_decode(q, kc, vc, seqlens, scale, 1, sink, W, block)
+    sa, _ = oracle.attn_decode(q, kc, vc, seqlens, scale, 0, sink, W, block)
+    ref = np.where(hm[None, :, None] == 1, fa, sa)
+    assert_close_attn(bits_of(o), ref, "per-head decode, group of 8")

@@ -63,7 +63,7 @@ def test_prefill_random_shape(ctx, seed):
 
 def _decode_case(seed):
     r = np.random.default_rng(seed)
-    G = int(r.choice([1, 2, 4]))
+    G = int(r.choice([1, 2, 3, 4, 5, 6, 7, 8]))
     Hkv = int(r.choice([1, 2, 3]))
     d = int(r.choice([64, 128]))
     block = int(r.choice([64, 128]))
