@@ -362,28 +362,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&bars[B_SF + 1]);
         umma_commit(&bars[B_KE + 0]);
       }
+      // The issue queue is shallow: this thread blocks in tcgen05.mma until
+      // about the previous MMA starts, so anything it does between two groups
+      // (even a wait that is already satisfied) idles the tensor core.  The
+      // operand waits therefore come first, where the thread waits for P0
+      // anyway, and the slot releases after the last group of the step.
       for (int j = 0; ok && j < n; ++j) {
         const int s = j & 1, sn = (j + 1) & 1;
         const bool more = j + 1 < n;
-        if (!mbar_wait(&bars[B_PF + 0], j & 1, a.st) ||
-            !mbar_wait(&bars[B_VF + s], (j >> 1) & 1, a.st)) { ok = false; break; }
+        if (!mbar_wait(&bars[B_VF + s], (j >> 1) & 1, a.st) ||
+            (more && !mbar_wait(&bars[B_KF + sn], ((j + 1) >> 1) & 1, a.st)) ||
+            !mbar_wait(&bars[B_PF + 0], j & 1, a.st)) { ok = false; break; }
         tc_fence_after();
         issue_pv(0, s, j > 0);
         if (more) {
-          if (!mbar_wait(&bars[B_KF + sn], ((j + 1) >> 1) & 1, a.st)) { ok = false; break; }
-          tc_fence_after();
           issue_s(0, sn);
           umma_commit(&bars[B_SF + 0]);
         }
         if (!mbar_wait(&bars[B_PF + 1], j & 1, a.st)) { ok = false; break; }
         tc_fence_after();
         issue_pv(1, s, j > 0);
-        umma_commit(&bars[B_VE + s]);
         if (more) {
           issue_s(1, sn);
           umma_commit(&bars[B_SF + 1]);
-          umma_commit(&bars[B_KE + sn]);
         }
+        umma_commit(&bars[B_VE + s]);
+        if (more) umma_commit(&bars[B_KE + sn]);
       }
       if (ok) umma_commit(&bars[B_OD]);
       // Every MMA issued by this thread is complete before TMEM is released.
