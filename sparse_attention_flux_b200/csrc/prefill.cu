@@ -53,6 +53,7 @@ struct PrefillArgs {
   int B, T, Hq, Hkv, G;
   int head_pair;     // 1: a CTA = one 128-row tile of two heads; 0: 256 rows of one head
   int nunit;         // CTA units along T: 128-row tiles (head pair) or 256-row pairs
+  int gchunk;        // kv groups whose units are scheduled together (divides Hkv)
   int nkt;           // 128-column key tiles along T
   int block;         // mask block: 64 or a multiple of 128
   int nqb;           // rows of the CSR
@@ -233,14 +234,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* nlist = reinterpret_cast<int*>(smem + L::NLIST);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Longest-first order: the last query rows carry the most causal work.
-  // Tile i (0, 1) holds rows [row0 + i * row_step, +128) of query head
-  // head0 + i * head_step.
-  const int hpu = a.head_pair ? a.Hq / 2 : a.Hq;   // head units per batch
-  const int per_unit = hpu * a.B;
-  const int unit = a.nunit - 1 - static_cast<int>(blockIdx.x) / per_unit;
-  const int rem = static_cast<int>(blockIdx.x) % per_unit;
-  const int b = rem / hpu, hu = rem % hpu;
+  // Order: sequence, then chunks of gchunk kv groups, then units longest
+  // first (the last query rows carry the most causal work), then the chunk's
+  // head units.  The CTAs in flight then read the K/V of gchunk groups only,
+  // which stays in L2 instead of being re-read from DRAM.  Tile i (0, 1)
+  // holds rows [row0 + i * row_step, +128) of query head head0 + i * head_step.
+  const int hpu = a.head_pair ? a.Hq / 2 : a.Hq;   // head units per sequence
+  const int cu = hpu / a.Hkv * a.gchunk;           // head units per chunk
+  const int per_chunk = cu * a.nunit;
+  const int per_seq = per_chunk * (a.Hkv / a.gchunk);
+  const int b = static_cast<int>(blockIdx.x) / per_seq;
+  const int rs_ = static_cast<int>(blockIdx.x) % per_seq;
+  const int chunk = rs_ / per_chunk, rc = rs_ % per_chunk;
+  const int unit = a.nunit - 1 - rc / cu;
+  const int hu = chunk * cu + rc % cu;
   const int row0 = unit * (a.head_pair ? kBM : 2 * kBM);          // first row of the unit
   const int nrow = a.head_pair ? kBM : 2 * kBM;                    // rows of the unit
   const int head0 = a.head_pair ? 2 * hu : hu, head_step = a.head_pair ? 1 : 0;
@@ -637,6 +644,15 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   a.head_pair = (a.G % 2 == 0 && p.head_mode == nullptr) ? 1 : 0;
   a.nunit = a.head_pair ? (p.T + kBM - 1) / kBM : (p.T + 2 * kBM - 1) / (2 * kBM);
   a.nkt = (p.T + kBN - 1) / kBN;
+  // As many kv groups per chunk (a divisor of Hkv) as keep their K and V
+  // within 72 MB, inside L2 beside the Q and O streams (measured: DRAM reads
+  // fall to the algorithmic bytes; 48 MB cost 1.4 %, 72 MB nothing).
+  {
+    const long long kv_bytes = 4LL * p.T * p.d;   // K + V of one group, bf16
+    a.gchunk = 1;
+    for (int gcand = p.Hkv; gcand > 1; --gcand)
+      if (p.Hkv % gcand == 0 && gcand * kv_bytes <= (72LL << 20)) { a.gchunk = gcand; break; }
+  }
   a.block = p.block;
   a.nqb = p.nqb;
   a.nkb = (p.T + p.block - 1) / p.block;
