@@ -13,6 +13,8 @@
 //     so no MMA or softmax is spent on a tile that only one of them sees; or
 //   a row pair (odd group size, or per-head routing): rows [256u, 256u + 256)
 //     of one query head, walking the union of the two tiles' lists.
+// CTAs are ordered per sequence, in chunks of kv groups whose K/V fit in L2,
+// longest unit first within a chunk.
 //
 // Per CTA (384 threads, warp-specialised):
 //   warp 0      TMA producer (Q0, Q1 once; K/V tiles into a 2-stage ring, K
@@ -22,7 +24,9 @@
 //                 S_i = Q_i K^T             (A, B from shared memory)
 //                 O_i += P_i V              (A = P_i from TMEM, B from smem)
 //               issued in the order S0 S1 | PV0 S0' PV1 S1' | ... so that the
-//               tensor core works on one tile while the other's softmax runs.
+//               tensor core works on one tile while the other's softmax runs;
+//               the issue queue is shallow, so the thread's barrier waits and
+//               slot releases sit outside the back-to-back MMA groups.
 //   warps 2, 3  idle.
 //   warps 4-7   softmax of Q0, warps 8-11 softmax of Q1: one query row per
 //               thread (= one TMEM lane); online softmax in the log2 domain;
