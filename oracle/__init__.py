@@ -11,7 +11,11 @@ arrays through ctypes.  bf16 tensors are passed as their raw 16-bit patterns
 (``numpy.uint16``), which the C code widens exactly to double.
 
 Each function cites the passage it follows in its C definition.  Pins:
-``tests/test_oracle.py``.  No function here is "parity unpinned".
+``tests/test_oracle.py`` and ``tests/test_block_select_oracle.py``.  One part is
+"parity unpinned" against the pages: the dynamic SA block selector
+(``block_scores``, ``select_blocks``), whose algorithm the pages do not give;
+it is pinned to brute force, closed forms and invariants of the reading stated
+in its C definition.
 """
 from __future__ import annotations
 
@@ -68,6 +72,8 @@ def lib() -> ctypes.CDLL:
             L.oracle_attn_probs.argtypes = [_u16p, _u16p, i, i, i, i, i, _vp, i, i, d, i, i, _f64p]
             L.oracle_attn_decode.argtypes = [_u16p, _u16p, _u16p, i, _i32p, i, i, i, i, i, i, i,
                                              i, d, _f64p, _vp]
+            L.oracle_block_scores.argtypes = [_u16p, _u16p, i, i, i, i, i, i, i, d, _f64p]
+            L.oracle_select_blocks.argtypes = [_f32p, i, f, i, _u8p]
             _lib = L
     return _lib
 
@@ -237,3 +243,33 @@ def attn_decode(q, k_cache, v_cache, seqlens, scale: float, mode: int, sink_bloc
     _check(lib().oracle_attn_decode(q, kc, vc, S_max, sl, B, Hq, Hkv, d, int(mode), sink_blocks,
                                     window_blocks, block, scale, o, _ptr(lse)), "attn_decode")
     return o, lse
+
+
+def block_scores(q, k, block: int, stride: int, scale: float) -> np.ndarray:
+    """Dynamic SA block selection, step 1 (reading stated in flux_oracle.c):
+    fp64 layer scores P [nb, nb] from strided antidiagonal logits; q uint16
+    [B, T, Hq, d], k uint16 [B, T, Hkv, d].  Row i sums to 1 over j <= i.
+    Parity unpinned against the pages."""
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    nr = (T + stride - 1) // stride
+    R = block // stride
+    nb = (nr + R - 1) // R
+    P = np.zeros((nb, nb), np.float64)
+    _check(lib().oracle_block_scores(q, k, B, T, Hq, Hkv, d, block, stride, scale, P),
+           "block_scores")
+    return P
+
+
+def select_blocks(P, tau: float, sink_blocks: int) -> np.ndarray:
+    """Dynamic SA block selection, step 2: the block mask uint8 [nb, nb] kept
+    from fp32 scores P (an fp64 P is rounded to fp32 first).  Parity unpinned
+    against the pages."""
+    P32 = np.ascontiguousarray(P, np.float32)
+    nb = P32.shape[0]
+    mask = np.zeros((nb, nb), np.uint8)
+    _check(lib().oracle_select_blocks(P32, nb, float(tau), int(sink_blocks), mask),
+           "select_blocks")
+    return mask

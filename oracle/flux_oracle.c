@@ -401,3 +401,154 @@ int oracle_attn_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_
     }
     return bad ? -1 : 0;
 }
+
+/*
+ * Dynamic SA block selection.  The pages name a block-sparse selector as the
+ * SA side's prior art (the checkpoint page's repository name
+ * "full_xattn_Qwen3-4B"; XAttention among the sparse methods in the UniSparse
+ * abstract on the page list) but give no algorithm.  The reading implemented
+ * here follows the published idea of that family -- score each block by
+ * antidiagonal sums over strided positions, then keep the fewest blocks whose
+ * score mass reaches a threshold -- with every detail fixed as follows:
+ *   strided positions r = 0 .. nr-1, nr = ceil(T / S): token rows r*S .. r*S+S-1,
+ *     a row >= T reading as a zero vector;
+ *   antidiagonal logit  z[r][c] = scale * sum_{k<S} q[r*S+k] . key[c*S+S-1-k],  c <= r;
+ *   block mass  E_h[i][j] = sum of exp(z[r][c]) over the strided rows r of query
+ *     block i and strided columns c of key block j (R = block / S of each), c <= r;
+ *   P_h[i][j] = E_h[i][j] / sum_{j' <= i} E_h[i][j']: the share of query block
+ *     i's antidiagonal attention mass that falls in key block j (head h of
+ *     sequence b, kv head h / (Hq/Hkv));
+ *   layer score  P[i][j] = mean over (b, h) of P_h[i][j].
+ * Parity unpinned against the pages (they print no algorithm); these
+ * functions are pinned to brute force, closed forms and invariants of the
+ * definition above.
+ */
+int oracle_block_scores(const uint16_t* q, const uint16_t* k, int B, int T, int Hq, int Hkv,
+                        int d, int block, int stride, double scale, double* P) {
+    if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || d < 1 || stride < 1 ||
+        block < stride || block % stride) return -1;
+    const int G = Hq / Hkv, S = stride, R = block / S;
+    const int nr = (T + S - 1) / S, nb = (nr + R - 1) / R;
+    const int nbh = B * Hq;
+    double* Ph = (double*)calloc((size_t)nbh * nb * nb, sizeof(double));
+    if (!Ph) return -1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double* qs = (double*)malloc(sizeof(double) * (size_t)R * S * d);   /* block i's rows */
+        double* ks = (double*)malloc(sizeof(double) * (size_t)S * d);       /* one strided col */
+        double* z = (double*)malloc(sizeof(double) * (size_t)R * nr);
+#pragma omp for schedule(dynamic, 1)
+        for (long long w = 0; w < (long long)nbh * nb; ++w) {
+            if (!qs || !ks || !z) {
+#pragma omp atomic write
+                bad = 1;
+                continue;
+            }
+            const int bh = (int)(w / nb), i = (int)(w % nb);
+            const int b = bh / Hq, h = bh % Hq, g = h / G;
+            const int r0 = i * R, r1 = r0 + R < nr ? r0 + R : nr;
+            /* the query rows of block i, widened (zero past T) */
+            for (int r = r0; r < r1; ++r)
+                for (int kk = 0; kk < S; ++kk) {
+                    const int t = r * S + kk;
+                    double* dst = qs + ((size_t)(r - r0) * S + kk) * d;
+                    for (int c = 0; c < d; ++c)
+                        dst[c] = t < T ? bf16_to_double(q[(((size_t)b * T + t) * Hq + h) * d + c]) : 0.0;
+                }
+            /* logits z[r][c] for c <= r, and their maximum */
+            double zmax = -INFINITY;
+            for (int cc = 0; cc < r1; ++cc) {
+                for (int kk = 0; kk < S; ++kk) {
+                    const int u = cc * S + S - 1 - kk;
+                    for (int c = 0; c < d; ++c)
+                        ks[(size_t)kk * d + c] =
+                            u < T ? bf16_to_double(k[(((size_t)b * T + u) * Hkv + g) * d + c]) : 0.0;
+                }
+                for (int r = r0; r < r1; ++r) {
+                    if (cc > r) continue;
+                    double acc = 0.0;
+                    for (int kk = 0; kk < S; ++kk) {
+                        const double* qa = qs + ((size_t)(r - r0) * S + kk) * d;
+                        const double* kb = ks + (size_t)kk * d;
+                        for (int c = 0; c < d; ++c) acc += qa[c] * kb[c];
+                    }
+                    acc *= scale;
+                    z[(size_t)(r - r0) * nr + cc] = acc;
+                    if (acc > zmax) zmax = acc;
+                }
+            }
+            /* block masses relative to exp(zmax), then their shares */
+            double* row = Ph + ((size_t)bh * nb + i) * nb;
+            double tot = 0.0;
+            for (int j = 0; j <= i; ++j) {
+                double e = 0.0;
+                for (int r = r0; r < r1; ++r)
+                    for (int cc = j * R; cc < (j + 1) * R && cc <= r; ++cc)
+                        e += exp(z[(size_t)(r - r0) * nr + cc] - zmax);
+                row[j] = e;
+                tot += e;
+            }
+            for (int j = 0; j <= i; ++j) row[j] /= tot;
+        }
+        free(qs);
+        free(ks);
+        free(z);
+    }
+    if (!bad) {
+        /* mean over (b, h), summed in a fixed order */
+        for (size_t e = 0; e < (size_t)nb * nb; ++e) {
+            double s = 0.0;
+            for (int bh = 0; bh < nbh; ++bh) s += Ph[(size_t)bh * nb * nb + e];
+            P[e] = s / nbh;
+        }
+    }
+    free(Ph);
+    return bad ? -1 : 0;
+}
+
+/*
+ * Selection from the layer scores (same reading as above): per query block
+ * i, the blocks j < sink_blocks (j <= i) and j = i are always kept; the other
+ * j <= i are taken in order of decreasing score (ties: smaller j first) while
+ * the running sum of the kept blocks' scores is below tau.  The scores and the
+ * running sum are fp32, summed in exactly this order (the forced blocks by
+ * ascending j, then the candidates as taken): the decision is an integer taken
+ * in the kernel's precision.
+ */
+int oracle_select_blocks(const float* P, int nb, float tau, int sink_blocks, uint8_t* mask) {
+    if (nb < 1 || sink_blocks < 0) return -1;
+    int* order = (int*)malloc(sizeof(int) * (size_t)nb);
+    if (!order) return -1;
+    memset(mask, 0, (size_t)nb * nb);
+    for (int i = 0; i < nb; ++i) {
+        const float* p = P + (size_t)i * nb;
+        uint8_t* m = mask + (size_t)i * nb;
+        float cum = 0.0f;
+        int n = 0;
+        for (int j = 0; j <= i; ++j) {
+            if (j < sink_blocks || j == i) {
+                m[j] = 1;
+                cum += p[j];
+            } else {
+                order[n++] = j;
+            }
+        }
+        /* insertion sort: decreasing score, then increasing j */
+        for (int a = 1; a < n; ++a) {
+            const int x = order[a];
+            int c = a - 1;
+            while (c >= 0 && (p[order[c]] < p[x] || (p[order[c]] == p[x] && order[c] > x))) {
+                order[c + 1] = order[c];
+                --c;
+            }
+            order[c + 1] = x;
+        }
+        for (int a = 0; a < n && cum < tau; ++a) {
+            m[order[a]] = 1;
+            cum += p[order[a]];
+        }
+    }
+    free(order);
+    return 0;
+}
