@@ -11,6 +11,7 @@
  *
  *   flux_route                 pool + MLP + hard threshold  -> layer_mode[L]
  *   flux_build_streaming_mask  sink + window block mask     -> mask[nqb][nkb]
+ *   flux_select_blocks         dynamic block mask from Q, K -> mask[nb][nb]
  *   flux_build_block_index     block mask                   -> CSR row_ptr/col
  *   flux_attn_prefill          one layer, FA or SA per layer_mode[layer]
  *   flux_attn_prefill_soft     r FA + (1 - r) SA, the training-time soft routing
@@ -127,6 +128,41 @@ int flux_route(flux_ctx* ctx, const uint16_t* hidden, int T, int Hd, int n_pool,
  *   The window counts the diagonal block.  sink_blocks >= 0, window_blocks >= 1. */
 int flux_build_streaming_mask(int nqb, int nkb, int sink_blocks, int window_blocks,
                               uint8_t* block_mask, flux_stream_t stream);
+
+/* Dynamic SA block selection: a block mask chosen from the layer's own Q and
+ * K.  The pages name a block-sparse selector for the SA side (the checkpoint
+ * page's repository name "full_xattn_Qwen3-4B"; XAttention among the sparse
+ * methods in the UniSparse abstract on the page list) but give no algorithm;
+ * this call implements a stated reading of that family's published idea
+ * (antidiagonal scores over strided positions, then the fewest blocks whose
+ * score mass reaches tau).  Parity against the pages is therefore unpinned;
+ * the definition below is the contract.  With S = stride, R = block / S,
+ * nr = ceil(T / S) strided positions and nb = ceil(T / block) blocks:
+ *   z[r][c]   = scale * sum_{k<S} q[rS+k] . key[cS+S-1-k] for c <= r < nr, per
+ *               (sequence b, query head h, kv head h / (Hq/Hkv)); rows >= T
+ *               read as zero;
+ *   P_h[i][j] = sum of exp(z) over strided rows r in [iR, iR+R) and columns c
+ *               in [jR, jR+R), c <= r, divided by that sum over all j <= i;
+ *   P[i][j]   = mean over (b, h) of P_h[i][j]  (block_score, fp32);
+ *   block_mask[i][j] = 1 for j < sink_blocks (j <= i) and j = i, and for the
+ *               other j <= i taken by decreasing P (ties: smaller j first)
+ *               while the fp32 sum of the kept blocks' P (forced blocks by
+ *               ascending j, then in the order taken) is below tau.
+ * One mask for the layer (all sequences and heads), the input of
+ * flux_build_block_index and of an SA prefill with the same block.
+ *   q [B, T, Hq, d], k [B, T, Hkv, d] bf16 in (16-byte aligned, contiguous).
+ *   block_mask [nb, nb] uint8 out; block_score [nb, nb] fp32 out (optional,
+ *   zero above the diagonal).
+ * Supported: d 64 or 128, block 128, stride 8 or 16, T <= 131072.  Uses
+ * flux_select_blocks_workspace_bytes() bytes of the ctx workspace.
+ * Errors: INVALID_ARG (null pointers, scale not finite and positive, tau
+ * negative or not finite, sink_blocks < 0, misaligned q/k), UNSUPPORTED
+ * (d, block, stride, T, Hq % Hkv), SHAPE (sizes, workspace too small). */
+size_t flux_select_blocks_workspace_bytes(int B, int T, int Hq, int Hkv, int stride);
+int flux_select_blocks(flux_ctx* ctx, const uint16_t* q, const uint16_t* k, int B, int T,
+                       int Hq, int Hkv, int d, int block, int stride, float scale, float tau,
+                       int sink_blocks, uint8_t* block_mask, float* block_score,
+                       flux_stream_t stream);
 
 /* Compressed block-index list of a block mask (the form the prefill kernel
  * walks, so that skipped blocks cost no memory traffic).

@@ -413,6 +413,63 @@ int flux_route(flux_ctx* c, const uint16_t* hidden, int T, int Hd, int n_pool, c
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_route: launch");
 }
 
+size_t flux_select_blocks_workspace_bytes(int B, int T, int Hq, int Hkv, int stride) {
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (stride != 8 && stride != 16))
+    return 0;
+  return flux::block_select_workspace_bytes(B, T, Hq, Hkv, stride);
+}
+
+int flux_select_blocks(flux_ctx* c, const uint16_t* q, const uint16_t* k, int B, int T, int Hq,
+                       int Hkv, int d, int block, int stride, float scale, float tau,
+                       int sink_blocks, uint8_t* block_mask, float* block_score,
+                       flux_stream_t stream) {
+  if (!c || !q || !k || !block_mask)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_select_blocks: null pointer argument");
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1)
+    return fail(FLUX_ERR_SHAPE, "flux_select_blocks: sizes must be positive");
+  if (d != 64 && d != 128)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_select_blocks: head_dim %d (supported: 64, 128)", d);
+  if (Hq % Hkv != 0)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_select_blocks: Hq %% Hkv != 0 (%d, %d)", Hq, Hkv);
+  if (block != 128 || (stride != 8 && stride != 16))
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_select_blocks: block %d stride %d (supported: "
+                "block 128, stride 8 or 16)", block, stride);
+  if ((T + block - 1) / block > flux::kSelectMaxBlocks)
+    return fail(FLUX_ERR_UNSUPPORTED, "flux_select_blocks: T %d above %d", T,
+                flux::kSelectMaxBlocks * block);
+  if (!(scale == scale) || scale <= 0.f || scale > 3.0e38f)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_select_blocks: scale must be finite and positive");
+  if (!(tau == tau) || tau < 0.f || tau > 3.0e38f || sink_blocks < 0)
+    return fail(FLUX_ERR_INVALID_ARG, "flux_select_blocks: tau must be finite and >= 0, "
+                "sink_blocks >= 0");
+  if (!aligned16(q) || !aligned16(k))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_select_blocks: q and k must be 16-byte aligned");
+  const size_t need = flux::block_select_workspace_bytes(B, T, Hq, Hkv, stride);
+  if (need > c->workspace_bytes)
+    return fail(FLUX_ERR_SHAPE, "flux_select_blocks: workspace %zu < %zu bytes",
+                c->workspace_bytes, need);
+  CUtensorMap tq, tk;
+  int rc;
+  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  flux::BlockSelectLaunch p;
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.d = d;
+  p.stride = stride;
+  p.scale = scale;
+  p.tau = tau;
+  p.sink_blocks = sink_blocks;
+  p.block_mask = block_mask;
+  p.block_score = block_score;
+  p.workspace = static_cast<float*>(c->workspace);
+  p.st = status_of(c);
+  const cudaError_t e = flux::launch_block_select(tq, tk, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_select_blocks: launch");
+}
+
 int flux_build_streaming_mask(int nqb, int nkb, int sink_blocks, int window_blocks,
                               uint8_t* block_mask, flux_stream_t stream) {
   if (!block_mask) return fail(FLUX_ERR_INVALID_ARG, "flux_build_streaming_mask: null mask");

@@ -91,6 +91,22 @@ struct RouteLaunch {
 size_t route_workspace_bytes(int Hd, int H1);
 cudaError_t launch_route(const RouteLaunch& p, cudaStream_t stream);
 
+// Dynamic SA block selection (strided antidiagonal scores, threshold selection).
+constexpr int kSelectMaxBlocks = 1024;   // query / key blocks of 128 tokens: T <= 131072
+struct BlockSelectLaunch {
+  int B, T, Hq, Hkv, d;
+  int stride;                // 8 or 16 (block 128)
+  float scale, tau;
+  int sink_blocks;
+  uint8_t* block_mask;       // [nb][nb] out
+  float* block_score;        // [nb][nb] out, optional
+  float* workspace;          // block_select_workspace_bytes()
+  DevStatus st;
+};
+size_t block_select_workspace_bytes(int B, int T, int Hq, int Hkv, int stride);
+cudaError_t launch_block_select(const CUtensorMap& tq, const CUtensorMap& tk,
+                                const BlockSelectLaunch& p, cudaStream_t stream);
+
 cudaError_t launch_ring_write(const uint16_t* k_src, const uint16_t* v_src, int n,
                               const int32_t* seqlens, int B, int Hkv, int d, uint16_t* k_ring,
                               uint16_t* v_ring, int sink, int window, int block, int* err,

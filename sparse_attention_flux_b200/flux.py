@@ -52,6 +52,9 @@ _SIGNATURES = {
     "flux_route": ([_vp, _vp, _i, _i, _i, _vp, _vp, _i, _vp, _vp, _i, _f, _vp, _vp, _vp], _i),
     "flux_build_streaming_mask": ([_i, _i, _i, _i, _vp, _vp], _i),
     "flux_build_block_index": ([_vp, _vp, _i, _i, _vp, _vp, _i, _vp], _i),
+    "flux_select_blocks": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _f, _i, _vp, _vp, _vp],
+                           _i),
+    "flux_select_blocks_workspace_bytes": ([_i, _i, _i, _i, _i], ctypes.c_size_t),
     "flux_attn_prefill": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp,
                            _i, _i, _f, _vp], _i),
     "flux_attn_decode": ([_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i, _i, _i,
@@ -216,6 +219,26 @@ class Context:
             raise ValueError("row_ptr needs nqb + 1 entries")
         _check(lib().flux_build_block_index(self._h, _ptr(block_mask), nqb, nkb, _ptr(row_ptr),
                                             _ptr(col), col.numel(), _stream(stream)))
+
+    def select_blocks(self, q, k, block_mask, scale: float, tau: float, sink_blocks: int = 0,
+                      stride: int = 8, block: int = 128, block_score=None, stream=None):
+        """flux_select_blocks: a dynamic SA block mask [nb, nb] from this layer's q, k."""
+        import torch
+        _need(q, torch.bfloat16, "q", self.device)
+        _need(k, torch.bfloat16, "k", self.device)
+        _need(block_mask, torch.uint8, "block_mask", self.device)
+        B, T, Hq, d = q.shape
+        Hkv = k.shape[2]
+        nb = (T + block - 1) // block
+        if block_mask.numel() < nb * nb:
+            raise ValueError("block_mask needs nb * nb entries")
+        if block_score is not None:
+            _need(block_score, torch.float32, "block_score", self.device)
+            if block_score.numel() < nb * nb:
+                raise ValueError("block_score needs nb * nb entries")
+        _check(lib().flux_select_blocks(self._h, _ptr(q), _ptr(k), B, T, Hq, Hkv, d, block,
+                                        stride, float(scale), float(tau), sink_blocks,
+                                        _ptr(block_mask), _ptr(block_score), _stream(stream)))
 
     # ------------------------------------------------------------------ attention
     def attn_prefill(self, q, k, v, o, scale: float, layer_mode=None, layer: int = 0,

@@ -93,3 +93,33 @@ def test_decode_family_host_checks_need_no_gpu(lib):
     # misaligned cache pointer
     assert lib.flux_attn_decode(ctx, P, ctypes.c_void_p(258), P, 64, P, P, None, 1, 2, 1, 64,
                                 None, 0, 1, 1, 64, 0.1, None) == flux.FLUX_ERR_INVALID_ARG
+
+
+def test_select_blocks_host_checks_need_no_gpu(lib):
+    """flux_select_blocks rejects bad arguments before any CUDA call."""
+    P = ctypes.c_void_p(256)
+    ctx = ctypes.c_void_p(4096)   # never dereferenced: the checks fail first
+    M = ctypes.c_void_p(512)
+    f = lib.flux_select_blocks
+    assert f(None, P, P, 1, 256, 2, 1, 64, 128, 8, 0.125, 0.9, 0, M, None, None) == \
+        flux.FLUX_ERR_INVALID_ARG
+    assert f(ctx, P, P, 1, 256, 2, 1, 96, 128, 8, 0.125, 0.9, 0, M, None, None) == \
+        flux.FLUX_ERR_UNSUPPORTED
+    assert f(ctx, P, P, 1, 256, 2, 1, 64, 64, 8, 0.125, 0.9, 0, M, None, None) == \
+        flux.FLUX_ERR_UNSUPPORTED
+    assert f(ctx, P, P, 1, 256, 2, 1, 64, 128, 4, 0.125, 0.9, 0, M, None, None) == \
+        flux.FLUX_ERR_UNSUPPORTED
+    assert f(ctx, P, P, 1, 200000, 2, 1, 64, 128, 8, 0.125, 0.9, 0, M, None, None) == \
+        flux.FLUX_ERR_UNSUPPORTED
+    assert f(ctx, P, P, 1, 256, 3, 2, 64, 128, 8, 0.125, 0.9, 0, M, None, None) == \
+        flux.FLUX_ERR_UNSUPPORTED
+    assert f(ctx, P, P, 1, 256, 2, 1, 64, 128, 8, float("nan"), 0.9, 0, M, None, None) == \
+        flux.FLUX_ERR_INVALID_ARG
+    assert f(ctx, P, P, 1, 256, 2, 1, 64, 128, 8, 0.125, -0.5, 0, M, None, None) == \
+        flux.FLUX_ERR_INVALID_ARG
+    assert f(ctx, ctypes.c_void_p(258), P, 1, 256, 2, 1, 64, 128, 8, 0.125, 0.9, 0, M, None,
+             None) == flux.FLUX_ERR_INVALID_ARG
+    # workspace: B * Hkv * nb * nb floats (4 query heads per CTA here)
+    nb = 32768 // 128
+    assert lib.flux_select_blocks_workspace_bytes(1, 32768, 32, 8, 8) == 8 * nb * nb * 4
+    assert lib.flux_select_blocks_workspace_bytes(1, 256, 3, 2, 8) == 0

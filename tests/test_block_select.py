@@ -1,0 +1,107 @@
+"""Dynamic SA block selection on the GPU against the oracle.
+
+The scores (fp32 on the GPU, fp64 in the oracle) are compared element by element;
+the mask is an integer decided from fp32 scores, so the oracle's selection is run
+on the GPU's own scores and must match bit for bit.  The selected mask then drives
+the CSR builder and SA prefill, compared with the oracle's attention under the same
+mask."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_flux_b200 import synth
+from sparse_attention_flux_b200.flux import Context
+from helpers import assert_close_attn, bits_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    with Context(0, 128 << 20) as c:
+        yield c
+
+
+def _select(ctx, q, k, stride, tau, sink):
+    dev = ctx.device
+    qt, kt = synth.torch_from_bits(q).to(dev), synth.torch_from_bits(k).to(dev)
+    T, d = q.shape[1], q.shape[3]
+    nb = (T + 127) // 128
+    mask = torch.full((nb, nb), 7, dtype=torch.uint8, device=dev)
+    score = torch.full((nb, nb), float("nan"), dtype=torch.float32, device=dev)
+    ctx.select_blocks(qt, kt, mask, 1 / math.sqrt(d), tau, sink, stride=stride, block_score=score)
+    ctx.check()
+    return mask.cpu().numpy(), score.cpu().numpy()
+
+
+CASES = [  # B, T, Hq, Hkv, d, stride, tau, sink
+    (1, 1024, 4, 2, 128, 8, 0.9, 1),
+    (2, 700, 6, 2, 64, 16, 0.8, 0),      # ragged T; 3 query heads per kv head
+    (1, 1500, 8, 1, 128, 8, 0.95, 2),    # 8 heads per kv head: two CTAs of four
+    (1, 128, 2, 2, 64, 8, 0.5, 0),       # a single block
+    (1, 3000, 5, 1, 64, 8, 0.9, 1),      # 5 heads per kv head: one per CTA
+    (1, 2049, 4, 1, 128, 16, 0.7, 1),    # one token past a block boundary
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_scores_and_mask_match_oracle(ctx, case):
+    B, T, Hq, Hkv, d, stride, tau, sink = case
+    q, k, _ = synth.attention_inputs(B, T, Hq, Hkv, d, seed=600 + T)
+    mask, score = _select(ctx, q, k, stride, tau, sink)
+    P = oracle.block_scores(q, k, 128, stride, 1 / math.sqrt(d))
+    nb = P.shape[0]
+    lower = np.tril(np.ones((nb, nb), bool))
+    err = np.abs(score.astype(np.float64) - P)
+    assert err[lower].max() <= 5e-5 + 1e-3 * P[lower].max(), f"{case}: score error {err.max()}"
+    assert np.all(score[~lower] == 0)
+    np.testing.assert_allclose(score.astype(np.float64).sum(axis=1), 1.0, atol=1e-4)
+    # the integer decision, taken by the oracle on the GPU's fp32 scores
+    np.testing.assert_array_equal(mask, oracle.select_blocks(score, tau, sink), err_msg=str(case))
+
+
+def test_planted_block_is_selected(ctx):
+    # Keys of block 3 are the antidiagonal partners of query block 9's rows times 4:
+    # block 3 takes almost all of query block 9's mass, far outside any local window.
+    T, Hq, Hkv, d, S = 1536, 2, 1, 64, 8
+    q, k, _ = synth.attention_inputs(1, T, Hq, Hkv, d, seed=21)
+    qf, kf = synth.bf16_bits_to_f32(q), synth.bf16_bits_to_f32(k)
+    R = 128 // S
+    for c in range(3 * R, 4 * R):
+        for kk in range(S):
+            kf[0, c * S + S - 1 - kk, 0] = 4.0 * (qf[0, 9 * 128 + kk, 0] + qf[0, 9 * 128 + kk, 1])
+    k = synth.to_bf16_bits(kf)
+    mask, score = _select(ctx, q, k, S, 0.5, 1)
+    assert np.argmax(score[9, :10]) == 3
+    assert list(np.nonzero(mask[9])[0]) == [0, 3, 9]
+
+
+def test_selected_mask_drives_sa_prefill(ctx):
+    B, T, Hq, Hkv, d = 1, 1900, 4, 2, 128
+    q, k, v = synth.attention_inputs(B, T, Hq, Hkv, d, seed=33)
+    dev = ctx.device
+    qt, kt, vt = (synth.torch_from_bits(x).to(dev) for x in (q, k, v))
+    nb = (T + 127) // 128
+    mask = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
+    ctx.select_blocks(qt, kt, mask, 1 / math.sqrt(d), 0.8, 1)
+    rp = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(nb * nb, dtype=torch.int32, device=dev)
+    ctx.build_block_index(mask, rp, col)
+    o = torch.full_like(qt, float("nan"))
+    lm = torch.tensor([0], dtype=torch.uint8, device=dev)
+    ctx.attn_prefill(qt, kt, vt, o, 1 / math.sqrt(d), layer_mode=lm, row_ptr=rp, col=col, block=128)
+    ctx.check()
+    m = mask.cpu().numpy()
+    assert m.sum() < np.tril(np.ones((nb, nb))).sum()   # something was skipped
+    ro, _ = oracle.attn_prefill(q, k, v, 1 / math.sqrt(d), block_mask=m, block=128)
+    assert_close_attn(bits_of(o), ro, "SA prefill over the selected mask")
+
+
+def test_deterministic(ctx):
+    q, k, _ = synth.attention_inputs(2, 2500, 8, 2, 128, seed=44)
+    m1, s1 = _select(ctx, q, k, 8, 0.9, 1)
+    m2, s2 = _select(ctx, q, k, 8, 0.9, 1)
+    assert np.array_equal(m1, m2) and np.array_equal(s1, s2)
