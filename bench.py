@@ -20,7 +20,9 @@ without an L2 flush.  On one GPU the line also carries, each timed in a few seco
 "prefill_36_layers" (the routed 36-layer prefill at T 65536: router, mask, CSR, 36
 layers reading their bits on the device) and "llama_3_1_8b" (32-layer shapes:
 prefill FA and SA layers at T 131072 for windows of 8/16/32 blocks; 32-layer decode
-at B 4, S 131072 for 0-100 % SA layers); --no-extended skips them.
+at B 4, S 131072 for 0-100 % SA layers) and "dynamic_sa" (flux_select_blocks on the
+layer's Q/K, the CSR build and SA prefill over the selected mask, and the planted needles'
+key blocks it keeps); --no-extended skips them.
 
 Every input is seeded and synthetic; every timed input (640 MB for prefill,
 17 GB of KV for decode) is larger than the 126 MB L2, so no flush is needed.
@@ -676,6 +678,69 @@ def llama_sweep(ctx, dev, seed):
     return out
 
 
+def dynamic_sa(ctx, wl, dev, reps=5):
+    """Dynamic SA block selection on the bench layer's own Q and K (flux_select_blocks:
+    strided antidiagonal block scores, stride 8, then the fewest blocks after the sink
+    and the diagonal whose score mass reaches tau 0.9), the CSR build and SA prefill
+    over the selected mask; the share of causal blocks kept; and how many of the
+    planted needles' key blocks the selected mask keeps for the needle rows, against
+    the streaming (sink + window) mask."""
+    import torch
+    nb, S, tau = wl.nb, 8, 0.9
+    mask = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
+    rp = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(nb * nb, dtype=torch.int32, device=dev)
+    o = torch.empty_like(wl.q)
+    lm = torch.zeros(1, dtype=torch.uint8, device=dev)
+    sel = lambda: ctx.select_blocks(wl.q, wl.k, mask, wl.scale, tau, SINK, stride=S)
+    idx = lambda: ctx.build_block_index(mask, rp, col)
+    att = lambda: ctx.attn_prefill(wl.q, wl.k, wl.v, o, wl.scale, layer_mode=lm, row_ptr=rp,
+                                   col=col, block=BLOCK)
+    for f in (sel, idx, att):
+        f()
+    ctx.check()
+
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / reps
+    sel_ms, idx_ms, att_ms = timed(sel), timed(idx), timed(att)
+    ctx.check()
+    m = mask.cpu().numpy().astype(np.int64)
+    stream_mask = wl.mask.cpu().numpy()
+    kept = int(m.sum())
+    pairs = (kept - int(np.trace(m))) * BLOCK * BLOCK + nb * BLOCK * (BLOCK + 1) // 2
+    flops_sa = 4.0 * D * pairs * HQ
+    nr = T // S
+    flops_sel = 2.0 * S * D * (nr * (nr + 1) / 2) * HQ
+    hit_dyn = hit_st = total = 0
+    for (_h, r, pos) in wl.needles:
+        i = r // BLOCK
+        for j in sorted(set(int(p) // BLOCK for p in pos)):
+            total += 1
+            hit_dyn += int(m[i, j])
+            hit_st += int(stream_mask[i, j])
+    return {
+        "how": "flux_select_blocks on the layer's Q/K (stride 8, tau 0.9, sink 1, block 128) -> "
+               "flux_build_block_index -> SA prefill over the selected mask; scores are a "
+               "reading of the strided-antidiagonal selector the pages name (parity unpinned "
+               "against the pages)",
+        "select_ms": round(sel_ms, 4),
+        "select_TFLOP/s": round(flops_sel / (sel_ms * 1e-3) / 1e12, 1),
+        "csr_ms": round(idx_ms, 4),
+        "sa_prefill_ms": round(att_ms, 4),
+        "sa_prefill_TFLOP/s": round(flops_sa / (att_ms * 1e-3) / 1e12, 1),
+        "kept_blocks": kept, "causal_blocks": nb * (nb + 1) // 2,
+        "kept_fraction": round(kept / (nb * (nb + 1) / 2), 4),
+        "needle_key_blocks_kept": {"selected_mask": hit_dyn, "streaming_mask": hit_st,
+                                   "of": total},
+    }
+
+
 def run_flux(args, rank, world, dev_index):
     import torch
     import torch.distributed as dist
@@ -771,6 +836,8 @@ def run_flux(args, rank, world, dev_index):
     soft_ms = s0.elapsed_time(s1) / 3
     soft_line = {"ms": round(soft_ms, 4), "TFLOP/s": round(wl.flops / (soft_ms * 1e-3) / 1e12, 1),
                  "note": "flux_attn_prefill_soft, r = 0.3: FA + SA passes, blended in the SA epilogue"}
+
+    dyn_line = dynamic_sa(ctx, wl, dev) if (world == 1 and not args.no_extended) else None
 
     h2d_bytes, d2h_bytes, launches = wl.h2d_bytes, wl.d2h_bytes, wl.launches * args.steps
     fa_avg = statistics.mean(fa_ms)
@@ -880,6 +947,7 @@ def run_flux(args, rank, world, dev_index):
                        "frac": round(sa_tflops / peak_t, 4)},
         "fa_prefill": {"TFLOP/s": round(fa_tflops, 1), "ms": round(fa_avg, 4)},
         "soft_prefill": soft_line,
+        **({"dynamic_sa": dyn_line} if dyn_line else {}),
         "router": {"step_router_us": round(router_us, 2), "router_36_layers_us": round(router36_us, 2),
                    "per_layer_us_36": round(router36_us / 36, 3),
                    "context": "pages: 0.20 ms per layer (hardware not stated)"},

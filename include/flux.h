@@ -153,7 +153,7 @@ int flux_build_streaming_mask(int nqb, int nkb, int sink_blocks, int window_bloc
  *   q [B, T, Hq, d], k [B, T, Hkv, d] bf16 in (16-byte aligned, contiguous).
  *   block_mask [nb, nb] uint8 out; block_score [nb, nb] fp32 out (optional,
  *   zero above the diagonal).
- * Supported: d 64 or 128, block 128, stride 8 or 16, T <= 131072.  Uses
+ * Supported: d 64 or 128, block 128, stride 8, T <= 131072.  Uses
  * flux_select_blocks_workspace_bytes() bytes of the ctx workspace.
  * Errors: INVALID_ARG (null pointers, scale not finite and positive, tau
  * negative or not finite, sink_blocks < 0, misaligned q/k), UNSUPPORTED

@@ -66,15 +66,16 @@ EncodeTiledFn encode_fn() {
 }
 
 // A bf16 tensor [d3][d2][d1][d0] (d0 innermost), boxes of box0 x 1 x box2 x 1
-// with the 128-byte swizzle; out-of-range rows read as zero.
+// with the 128-byte swizzle; out-of-range rows read as zero.  With step2 > 1 a
+// box takes every step2-th d2 row of its box2-row span (box2 / step2 rows).
 int make_map_4d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                uint64_t d3, uint32_t box0, uint32_t box2) {
+                uint64_t d3, uint32_t box0, uint32_t box2, uint32_t step2 = 1) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(FLUX_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   const cuuint64_t gdim[4] = {d0, d1, d2, d3};
   const cuuint64_t gstride[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
   const cuuint32_t box[4] = {box0, 1, box2, 1};
-  const cuuint32_t estride[4] = {1, 1, 1, 1};
+  const cuuint32_t estride[4] = {1, 1, step2, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gdim,
                          gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -414,8 +415,7 @@ int flux_route(flux_ctx* c, const uint16_t* hidden, int T, int Hd, int n_pool, c
 }
 
 size_t flux_select_blocks_workspace_bytes(int B, int T, int Hq, int Hkv, int stride) {
-  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (stride != 8 && stride != 16))
-    return 0;
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || stride != 8) return 0;
   return flux::block_select_workspace_bytes(B, T, Hq, Hkv, stride);
 }
 
@@ -431,9 +431,9 @@ int flux_select_blocks(flux_ctx* c, const uint16_t* q, const uint16_t* k, int B,
     return fail(FLUX_ERR_UNSUPPORTED, "flux_select_blocks: head_dim %d (supported: 64, 128)", d);
   if (Hq % Hkv != 0)
     return fail(FLUX_ERR_UNSUPPORTED, "flux_select_blocks: Hq %% Hkv != 0 (%d, %d)", Hq, Hkv);
-  if (block != 128 || (stride != 8 && stride != 16))
+  if (block != 128 || stride != 8)
     return fail(FLUX_ERR_UNSUPPORTED, "flux_select_blocks: block %d stride %d (supported: "
-                "block 128, stride 8 or 16)", block, stride);
+                "block 128, stride 8)", block, stride);
   if ((T + block - 1) / block > flux::kSelectMaxBlocks)
     return fail(FLUX_ERR_UNSUPPORTED, "flux_select_blocks: T %d above %d", T,
                 flux::kSelectMaxBlocks * block);
@@ -450,8 +450,10 @@ int flux_select_blocks(flux_ctx* c, const uint16_t* q, const uint16_t* k, int B,
                 c->workspace_bytes, need);
   CUtensorMap tq, tk;
   int rc;
-  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128)) != FLUX_OK) return rc;
+  // Strided boxes: each load brings the rows of one antidiagonal offset, so the
+  // strided positions are consecutive rows in shared memory.
+  if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128, stride)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128, stride)) != FLUX_OK) return rc;
   flux::BlockSelectLaunch p;
   p.B = B;
   p.T = T;

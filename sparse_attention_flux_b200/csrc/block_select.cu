@@ -16,10 +16,13 @@
 //   block_score_kernel: one CTA per (sequence, kv head, chunk of up to four
 //     query heads, query block i), query blocks longest first.  TMA brings
 //     the chunk's Q tiles once and the K tile of every key block j <= i
-//     through a 2-stage ring; one warp per query head computes the R x R
-//     strided logits of (i, j) as 16x8x16 warp MMAs -- the antidiagonal
-//     pairing is only a row permutation of the ldmatrix addresses into the
-//     128-byte swizzled tiles -- and reduces them to the block's log-sum-exp.
+//     through a 2-stage ring, each tile as S strided boxes: box kk holds the
+//     R rows kk, kk + S, ... (K: S-1-kk, 2S-1-kk, ...), so strided position r
+//     is row r of every box and an ldmatrix over 8 positions touches 8
+//     different swizzle phases (rows S apart in one box would all share one:
+//     an 8-way bank conflict).  One warp per query head computes the R x R
+//     strided logits of (i, j) as 16x8x16 warp MMAs and reduces them to the
+//     block's log-sum-exp.
 //     At the end each head's shares are summed over the chunk into a
 //     per-chunk partial row.  Bound: the warp MMAs' issue (K tiles come from
 //     L2: the G heads of a kv group share them).
@@ -39,6 +42,8 @@ constexpr int kBox = 128 * 128;            // one 128-row x 64-channel swizzled 
 constexpr int kMaxHeads = 4;               // query heads per score CTA
 constexpr int kScoreThreads = 32 * (kMaxHeads + 1);
 constexpr int kSelectThreads = 256;
+// Stride of the strided positions: the TMA traversal stride, at most 8.
+constexpr int kStride = 8;
 
 struct ScoreArgs {
   int B, T, Hq, Hkv, G, hc;   // hc: query heads per CTA (divides G, <= kMaxHeads)
@@ -51,26 +56,29 @@ struct ScoreArgs {
 template <int D>
 struct ScoreSmem {
   static constexpr int CH = D / 64;
-  static constexpr int Q = 0;                              // [kMaxHeads][CH] boxes
-  static constexpr int K = Q + kMaxHeads * CH * kBox;      // [2 stages][CH]
+  // A tile (128 rows x D) = S strided boxes of R rows per 64-channel chunk,
+  // [kk][chunk][R rows x 128 B]: CH * kBox bytes whatever the stride.
+  static constexpr int Q = 0;                              // [kMaxHeads] tiles
+  static constexpr int K = Q + kMaxHeads * CH * kBox;      // [2 stages] tiles
   static constexpr int LSE = K + 2 * CH * kBox;            // f32 [kMaxHeads][nb]
   static int total(int nb) { return LSE + kMaxHeads * nb * 4 + 8 * 8 + 1024; }
 };
 
-// Shared-memory address of channel chunk uu (16 bytes) of row t in a tile of
-// CH boxes written by TMA with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t swz(uint32_t base, int t, int uu) {
-  return base + (uu >> 3) * kBox + t * 128 + (((uu & 7) ^ (t & 7)) << 4);
+// Shared-memory address of channel chunk uu (16 bytes) of strided row r in
+// box kk of a tile of strided boxes (R rows each, 128-byte swizzle).
+template <int R, int CH>
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int kk, int r, int uu) {
+  return tile + (kk * CH + (uu >> 3)) * (R * 128) + r * 128 + (((uu & 7) ^ (r & 7)) << 4);
 }
 
-template <int D, int S>
+template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     block_score_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
   using L = ScoreSmem<D>;
   constexpr int CH = L::CH;
-  constexpr int R = kTile / S;               // strided positions per block: 16 or 8
-  static_assert(R == 16 || R == 8, "stride 8 or 16");
+  constexpr int S = kStride;
+  constexpr int R = kTile / S;               // strided positions per block: 16 = one m16 tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -101,8 +109,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     tma_prefetch_desc(&tm_k);
     mbar_arrive_expect_tx(qbar, a.hc * CH * kBox);
     for (int w = 0; w < a.hc; ++w)
-      for (int c = 0; c < CH; ++c)
-        tma_load_4d(&tm_q, qbar, smem + L::Q + (w * CH + c) * kBox, c * 64, head0 + w, i * kTile, b);
+      for (int kk = 0; kk < S; ++kk)
+        for (int c = 0; c < CH; ++c)
+          tma_load_4d(&tm_q, qbar, smem + L::Q + w * CH * kBox + (kk * CH + c) * (R * 128),
+                      c * 64, head0 + w, i * kTile + kk, b);
   }
   __syncthreads();
 
@@ -114,8 +124,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         const int s = j & 1;
         if (j >= 2 && !mbar_wait(&empty[s], ((j >> 1) - 1) & 1, a.st)) break;
         mbar_arrive_expect_tx(&full[s], CH * kBox);
-        for (int c = 0; c < CH; ++c)
-          tma_load_4d(&tm_k, &full[s], smem + L::K + (s * CH + c) * kBox, c * 64, g, j * kTile, b);
+        for (int kk = 0; kk < S; ++kk)
+          for (int c = 0; c < CH; ++c)
+            tma_load_4d(&tm_k, &full[s], smem + L::K + s * CH * kBox + (kk * CH + c) * (R * 128),
+                        c * 64, g, j * kTile + S - 1 - kk, b);
         issued = j + 1;
       }
       mbar_drain(qbar, 0);
@@ -127,29 +139,26 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const int mi = lane >> 3, rr = lane & 7;     // ldmatrix: matrix, row within it
     const int gq = lane >> 2, tq = lane & 3;     // mma fragment: row group, column pair
     const uint32_t qbase = smem_u32(smem + L::Q + warp * CH * kBox);
-    // A rows: strided row ra (0..R-1); with R = 8 rows 8..15 repeat 0..7 and are zeroed.
-    const int ra = R == 16 ? ((mi & 1) << 3) + rr : rr;
-    // B rows: strided column cb of the n-tile; with R = 8 only n-tile 0 is used.
-    const int cb = R == 16 ? ((mi >> 1) << 3) + rr : rr;
+    const int ra = ((mi & 1) << 3) + rr;         // A: strided row of this lane's matrix row
+    const int cb = ((mi >> 1) << 3) + rr;        // B: strided column (two n-tiles of 8)
     float* my_lse = lse + warp * a.nb;
     bool ok = mbar_wait(qbar, 0, a.st);
     for (int j = 0; ok && j <= i; ++j) {
       const int s = j & 1;
       if (!mbar_wait(&full[s], (j >> 1) & 1, a.st)) { ok = false; break; }
       const uint32_t kbase = smem_u32(smem + L::K + s * CH * kBox);
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // Two partial sums per n-tile (even / odd channel steps) halve the
+      // dependent MMA chains.
+      float acc[2][2][4] = {};
 #pragma unroll 1
       for (int kk = 0; kk < S; ++kk) {
-        const int ta = ra * S + kk;                 // query token row of the A row
-        const int ub = cb * S + S - 1 - kk;         // key token row of the B row
 #pragma unroll
         for (int dc = 0; dc < D / 16; ++dc) {
           uint32_t af[4], b00, b01, b10, b11;
-          ldmatrix_x4(swz(qbase, ta, dc * 2 + (mi >> 1)), af[0], af[1], af[2], af[3]);
-          ldmatrix_x4(swz(kbase, ub, dc * 2 + (mi & 1)), b00, b01, b10, b11);
-          if (R == 8) af[1] = af[3] = 0u;
-          mma_bf16_16816(acc[0], af, b00, b01);
-          if (R == 16) mma_bf16_16816(acc[1], af, b10, b11);
+          ldmatrix_x4(swz<R, CH>(qbase, kk, ra, dc * 2 + (mi >> 1)), af[0], af[1], af[2], af[3]);
+          ldmatrix_x4(swz<R, CH>(kbase, kk, cb, dc * 2 + (mi & 1)), b00, b01, b10, b11);
+          mma_bf16_16816(acc[0][dc & 1], af, b00, b01);
+          mma_bf16_16816(acc[1][dc & 1], af, b10, b11);
         }
       }
       __syncwarp();
@@ -163,8 +172,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         for (int e = 0; e < 4; ++e) {
           const int r = gq + (e >> 1) * 8, c = nt * 8 + 2 * tq + (e & 1);
           const int rg = i * R + r, cg = j * R + c;
-          const bool valid = r < R && c < R && cg <= rg && rg < a.nr && cg < a.nr;
-          const float v = valid ? acc[nt][e] * a.scale_log2 : -INFINITY;
+          const bool valid = cg <= rg && rg < a.nr && cg < a.nr;
+          const float v = valid ? (acc[nt][0][e] + acc[nt][1][e]) * a.scale_log2 : -INFINITY;
           z[nt * 4 + e] = v;
           m = fmaxf(m, v);
         }
@@ -261,13 +270,13 @@ __global__ void __launch_bounds__(kSelectThreads)
   }
 }
 
-template <int D, int S>
+template <int D>
 cudaError_t launch_scores_t(const CUtensorMap& tq, const CUtensorMap& tk, const ScoreArgs& a,
                             cudaStream_t stream) {
   const int smem = ScoreSmem<D>::total(a.nb);
-  cudaFuncSetAttribute(block_score_kernel<D, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaFuncSetAttribute(block_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const unsigned grid = static_cast<unsigned>(a.nb) * a.B * a.Hkv * (a.G / a.hc);
-  block_score_kernel<D, S><<<grid, kScoreThreads, smem, stream>>>(tq, tk, a);
+  block_score_kernel<D><<<grid, kScoreThreads, smem, stream>>>(tq, tk, a);
   return cudaGetLastError();
 }
 
@@ -301,11 +310,9 @@ cudaError_t launch_block_select(const CUtensorMap& tq, const CUtensorMap& tk,
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.partial = p.workspace;
   a.st = p.st;
-  cudaError_t e;
-  if (p.d == 64)
-    e = p.stride == 8 ? launch_scores_t<64, 8>(tq, tk, a, stream) : launch_scores_t<64, 16>(tq, tk, a, stream);
-  else
-    e = p.stride == 8 ? launch_scores_t<128, 8>(tq, tk, a, stream) : launch_scores_t<128, 16>(tq, tk, a, stream);
+  if (p.stride != kStride) return cudaErrorInvalidValue;
+  const cudaError_t e = p.d == 64 ? launch_scores_t<64>(tq, tk, a, stream)
+                                  : launch_scores_t<128>(tq, tk, a, stream);
   if (e != cudaSuccess) return e;
   int n2 = 1;
   while (n2 < a.nb) n2 <<= 1;

@@ -95,7 +95,7 @@ cudaError_t launch_route(const RouteLaunch& p, cudaStream_t stream);
 constexpr int kSelectMaxBlocks = 1024;   // query / key blocks of 128 tokens: T <= 131072
 struct BlockSelectLaunch {
   int B, T, Hq, Hkv, d;
-  int stride;                // 8 or 16 (block 128)
+  int stride;                // 8 (block 128)
   float scale, tau;
   int sink_blocks;
   uint8_t* block_mask;       // [nb][nb] out

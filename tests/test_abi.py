@@ -107,7 +107,7 @@ def test_select_blocks_host_checks_need_no_gpu(lib):
         flux.FLUX_ERR_UNSUPPORTED
     assert f(ctx, P, P, 1, 256, 2, 1, 64, 64, 8, 0.125, 0.9, 0, M, None, None) == \
         flux.FLUX_ERR_UNSUPPORTED
-    assert f(ctx, P, P, 1, 256, 2, 1, 64, 128, 4, 0.125, 0.9, 0, M, None, None) == \
+    assert f(ctx, P, P, 1, 256, 2, 1, 64, 128, 16, 0.125, 0.9, 0, M, None, None) == \
         flux.FLUX_ERR_UNSUPPORTED
     assert f(ctx, P, P, 1, 200000, 2, 1, 64, 128, 8, 0.125, 0.9, 0, M, None, None) == \
         flux.FLUX_ERR_UNSUPPORTED

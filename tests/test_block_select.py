@@ -39,11 +39,11 @@ def _select(ctx, q, k, stride, tau, sink):
 
 CASES = [  # B, T, Hq, Hkv, d, stride, tau, sink
     (1, 1024, 4, 2, 128, 8, 0.9, 1),
-    (2, 700, 6, 2, 64, 16, 0.8, 0),      # ragged T; 3 query heads per kv head
+    (2, 700, 6, 2, 64, 8, 0.8, 0),       # ragged T; 3 query heads per kv head
     (1, 1500, 8, 1, 128, 8, 0.95, 2),    # 8 heads per kv head: two CTAs of four
     (1, 128, 2, 2, 64, 8, 0.5, 0),       # a single block
     (1, 3000, 5, 1, 64, 8, 0.9, 1),      # 5 heads per kv head: one per CTA
-    (1, 2049, 4, 1, 128, 16, 0.7, 1),    # one token past a block boundary
+    (1, 2049, 4, 1, 128, 8, 0.7, 1),     # one token past a block boundary
 ]
 
 
