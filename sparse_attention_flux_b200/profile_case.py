@@ -4,6 +4,7 @@
     python -m sparse_attention_flux_b200.profile_case decode --mode sa --B 4 --S 32768
     python -m sparse_attention_flux_b200.profile_case decode --mode ring --B 16 --S 131072
     python -m sparse_attention_flux_b200.profile_case append --mode ring --B 16 --S 131072
+    python -m sparse_attention_flux_b200.profile_case select --T 32768
 
 Inputs are seeded N(0, 1) bf16 drawn on the device; nothing is checked here
 (the test suite does that).  Prints the CUDA-event time per launch.
@@ -21,7 +22,7 @@ from sparse_attention_flux_b200.flux import Context
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["prefill", "decode", "route", "append"])
+    ap.add_argument("kernel", choices=["prefill", "decode", "route", "append", "select"])
     ap.add_argument("--mode", choices=["fa", "sa", "ring"], default="fa",
                     help="ring: SA decode / append over the compact sink + window cache")
     ap.add_argument("--B", type=int, default=1)
@@ -77,6 +78,13 @@ def main() -> None:
             run = lambda: ctx.attn_decode(q, kc, vc, sl, o, scale, layer_mode=mode,
                                           sink_blocks=args.sink, window_blocks=args.window,
                                           block=args.block)
+    elif args.kernel == "select":
+        B, T = args.B, args.T
+        q = synth.torch_normal_bf16((B, T, args.Hq, args.d), 1, dev)
+        k = synth.torch_normal_bf16((B, T, args.Hkv, args.d), 2, dev)
+        nb = (T + 127) // 128
+        m = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
+        run = lambda: ctx.select_blocks(q, k, m, scale, 0.9, args.sink, stride=8)
     else:
         T, Hd, H1, L = args.T, 2560, 512, 36
         hidden = synth.torch_normal_bf16((T, Hd), 1, dev)
