@@ -24,8 +24,10 @@
 //     strided logits of (i, j) as 16x8x16 warp MMAs and reduces them to the
 //     block's log-sum-exp.
 //     At the end each head's shares are summed over the chunk into a
-//     per-chunk partial row.  Bound: the warp MMAs' issue (K tiles come from
-//     L2: the G heads of a kv group share them).
+//     per-chunk partial row.  Bound: the latency of each warp's dependent
+//     ldmatrix -> mma chain, with four compute warps per SM (the Q tiles of
+//     four heads fill most of shared memory); the K tiles come from L2, shared
+//     by the heads of a kv group.
 //   block_select_kernel: one CTA per query block: the partial rows summed in
 //     a fixed order, a bitonic sort of the candidates (score descending, block
 //     ascending) and one thread's sequential fp32 running sum decide the kept
