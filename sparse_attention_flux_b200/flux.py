@@ -220,6 +220,11 @@ class Context:
         _check(lib().flux_build_block_index(self._h, _ptr(block_mask), nqb, nkb, _ptr(row_ptr),
                                             _ptr(col), col.numel(), _stream(stream)))
 
+    def select_blocks_workspace_bytes(self, B: int, T: int, Hq: int, Hkv: int,
+                                      stride: int = 8) -> int:
+        """Bytes of ctx workspace flux_select_blocks needs (0 for unsupported sizes)."""
+        return int(lib().flux_select_blocks_workspace_bytes(B, T, Hq, Hkv, stride))
+
     def select_blocks(self, q, k, block_mask, scale: float, tau: float, sink_blocks: int = 0,
                       stride: int = 8, block: int = 128, block_score=None, stream=None):
         """flux_select_blocks: a dynamic SA block mask [nb, nb] from this layer's q, k."""
