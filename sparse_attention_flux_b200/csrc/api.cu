@@ -451,9 +451,10 @@ int flux_select_blocks(flux_ctx* c, const uint16_t* q, const uint16_t* k, int B,
   CUtensorMap tq, tk;
   int rc;
   // Strided boxes: each load brings the rows of one antidiagonal offset, so the
-  // strided positions are consecutive rows in shared memory.
+  // strided positions are consecutive rows in shared memory (Q: 16 rows of one
+  // block; K: 32 rows spanning two blocks).
   if ((rc = make_map_4d(&tq, q, d, Hq, T, B, 64, 128, stride)) != FLUX_OK) return rc;
-  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 128, stride)) != FLUX_OK) return rc;
+  if ((rc = make_map_4d(&tk, k, d, Hkv, T, B, 64, 256, stride)) != FLUX_OK) return rc;
   flux::BlockSelectLaunch p;
   p.B = B;
   p.T = T;

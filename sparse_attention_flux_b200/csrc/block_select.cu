@@ -15,19 +15,19 @@
 // Two kernels:
 //   block_score_kernel: one CTA per (sequence, kv head, chunk of up to four
 //     query heads, query block i), query blocks longest first.  TMA brings
-//     the chunk's Q tiles once and the K tile of every key block j <= i
-//     through a 2-stage ring, each tile as S strided boxes: box kk holds the
-//     R rows kk, kk + S, ... (K: S-1-kk, 2S-1-kk, ...), so strided position r
-//     is row r of every box and an ldmatrix over 8 positions touches 8
-//     different swizzle phases (rows S apart in one box would all share one:
-//     an 8-way bank conflict).  One warp per query head computes the R x R
-//     strided logits of (i, j) as 16x8x16 warp MMAs and reduces them to the
-//     block's log-sum-exp.
-//     At the end each head's shares are summed over the chunk into a
-//     per-chunk partial row.  Bound: the latency of each warp's dependent
-//     ldmatrix -> mma chain, with four compute warps per SM (the Q tiles of
-//     four heads fill most of shared memory); the K tiles come from L2, shared
-//     by the heads of a kv group.
+//     the chunk's Q once and the K tile of every key block j <= i through a
+//     2-stage ring, each as 8 strided boxes (traversal stride 8): box kk holds
+//     the 16 rows kk, kk + 8, ... of Q (for K: 7-kk, 15-kk, ...), so the
+//     strided positions are consecutive rows and the antidiagonal pairing is
+//     the choice of box.  Q is the resident A operand of one tcgen05 MMA chain
+//     per key block: M 64 = four heads x 16 strided positions, N 16 strided
+//     key positions, K = 8 d (64 MMAs of K 16 at d 128), accumulated in a
+//     double-buffered TMEM tile; four epilogue warps (one per head, the
+//     head's rows being the first 16 lanes of its TMEM quarter) reduce each
+//     tile to the block's log-sum-exp while the next block's MMAs run, and
+//     at the end each head's shares are summed over the chunk into a
+//     per-chunk partial row.  Bound: the K tiles' stream from L2 (the heads
+//     of a kv group share them through the CTA).
 //   block_select_kernel: one CTA per query block: the partial rows summed in
 //     a fixed order, a bitonic sort of the candidates (score descending, block
 //     ascending) and one thread's sequential fp32 running sum decide the kept
@@ -40,9 +40,8 @@ namespace flux {
 namespace {
 
 constexpr int kTile = 128;                 // query / key block, tokens
-constexpr int kBox = 128 * 128;            // one 128-row x 64-channel swizzled box
 constexpr int kMaxHeads = 4;               // query heads per score CTA
-constexpr int kScoreThreads = 32 * (kMaxHeads + 1);
+constexpr int kScoreThreads = 32 * 6;      // K producer, MMA issuer, four epilogue warps
 constexpr int kSelectThreads = 256;
 // Stride of the strided positions: the TMA traversal stride, at most 8.
 constexpr int kStride = 8;
@@ -55,23 +54,24 @@ struct ScoreArgs {
   DevStatus st;
 };
 
+constexpr int kGroup = 8;                  // key blocks per MMA tile: M = 128 strided keys
+constexpr int kStages = 4;                 // K chunk ring
+
 template <int D>
 struct ScoreSmem {
   static constexpr int CH = D / 64;
-  // A tile (128 rows x D) = S strided boxes of R rows per 64-channel chunk,
-  // [kk][chunk][R rows x 128 B]: CH * kBox bytes whatever the stride.
-  static constexpr int Q = 0;                              // [kMaxHeads] tiles
-  static constexpr int K = Q + kMaxHeads * CH * kBox;      // [2 stages] tiles
-  static constexpr int LSE = K + 2 * CH * kBox;            // f32 [kMaxHeads][nb]
-  static int total(int nb) { return LSE + kMaxHeads * nb * 4 + 8 * 8 + 1024; }
+  static constexpr int QROWS = kMaxHeads * 16;   // MMA N: four heads x 16 strided rows
+  // Q (resident B operand): [kk][chunk][64 rows x 128 B].  K chunk (A operand, ring):
+  // [128 rows x 128 B] = one antidiagonal offset kk and one 64-channel chunk of 8 key
+  // blocks.  Both 128-byte swizzled, 8-row groups 1 KB apart.
+  static constexpr int Q = 0;
+  static constexpr int Q_BYTES = kStride * CH * QROWS * 128;   // CH * 64 KB
+  static constexpr int KC = Q + Q_BYTES;
+  static constexpr int KC_BYTES = kGroup * 16 * 128;           // 16 KB
+  static constexpr int LSE = KC + kStages * KC_BYTES;          // f32 [kMaxHeads][nb]
+  __host__ __device__ static int bars(int nb) { return LSE + kMaxHeads * nb * 4; }
+  __host__ __device__ static int total(int nb) { return bars(nb) + 16 * 8 + 1024; }
 };
-
-// Shared-memory address of channel chunk uu (16 bytes) of strided row r in
-// box kk of a tile of strided boxes (R rows each, 128-byte swizzle).
-template <int R, int CH>
-__device__ __forceinline__ uint32_t swz(uint32_t tile, int kk, int r, int uu) {
-  return tile + (kk * CH + (uu >> 3)) * (R * 128) + r * 128 + (((uu & 7) ^ (r & 7)) << 4);
-}
 
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 1)
@@ -80,15 +80,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   using L = ScoreSmem<D>;
   constexpr int CH = L::CH;
   constexpr int S = kStride;
-  constexpr int R = kTile / S;               // strided positions per block: 16 = one m16 tile
+  constexpr int R = kTile / S;               // 16 strided positions per block
+  constexpr int NCHUNK = S * CH;             // K chunks per group (K = 8 d in 64-channel steps)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   float* lse = reinterpret_cast<float*>(smem + L::LSE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::LSE + kMaxHeads * a.nb * 4);
-  uint64_t* full = bars;         // [2]
-  uint64_t* empty = bars + 2;    // [2]
-  uint64_t* qbar = bars + 4;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars(a.nb));
+  uint64_t* full = bars;                  // [kStages] K chunk landed
+  uint64_t* empty = bars + kStages;       // [kStages] K chunk read by its MMAs
+  uint64_t* dfull = bars + 2 * kStages;   // [2] accumulator tile written
+  uint64_t* dfree = dfull + 2;            // [2] accumulator tile read by the epilogue warps
+  uint64_t* qbar = dfull + 4;
+  uint64_t* drain = dfull + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dfull + 6);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nchunk = a.G / a.hc;
@@ -99,99 +104,151 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int g = (rem / nchunk) % a.Hkv;
   const int hc = rem % nchunk;
   const int head0 = g * a.G + hc * a.hc;
+  const int ngroups = i / kGroup + 1;        // key blocks 0..i in groups of 8
 
+  // A chunk of fewer than four heads: the absent heads' rows of Q are zero.
+  if (a.hc < kMaxHeads) {
+    const int per_box = (kMaxHeads - a.hc) * 16 * 128 / 16;   // uint4 per (kk, chunk)
+    for (int idx = threadIdx.x; idx < NCHUNK * per_box; idx += blockDim.x) {
+      const int box = idx / per_box, off = idx % per_box;
+      reinterpret_cast<uint4*>(smem + L::Q + box * (L::QROWS * 128) + a.hc * 16 * 128)[off] =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
   if (threadIdx.x == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    mbar_init(&empty[0], a.hc);
-    mbar_init(&empty[1], a.hc);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&dfull[s], 1);
+      mbar_init(&dfree[s], 4);
+    }
     mbar_init(qbar, 1);
+    mbar_init(drain, 1);
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
-    mbar_arrive_expect_tx(qbar, a.hc * CH * kBox);
+    mbar_arrive_expect_tx(qbar, a.hc * NCHUNK * 16 * 128);
     for (int w = 0; w < a.hc; ++w)
       for (int kk = 0; kk < S; ++kk)
         for (int c = 0; c < CH; ++c)
-          tma_load_4d(&tm_q, qbar, smem + L::Q + w * CH * kBox + (kk * CH + c) * (R * 128),
+          tma_load_4d(&tm_q, qbar, smem + L::Q + (kk * CH + c) * (L::QROWS * 128) + w * 16 * 128,
                       c * 64, head0 + w, i * kTile + kk, b);
   }
+  if (warp == 1) tmem_alloc(tmem_slot, 128);
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
 
-  if (warp == kMaxHeads) {
+  if (warp == 0) {
     // ------------------------------------------------------------ K producer
+    // Chunk t = (group, kk, channel chunk): 4 boxes of 32 strided rows, each
+    // spanning two key blocks (rows 7-kk, 15-kk, ... of key blocks 2q, 2q+1).
     if (lane == 0) {
+      const int total = ngroups * NCHUNK;
       int issued = 0;
-      for (int j = 0; j <= i; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&empty[s], ((j >> 1) - 1) & 1, a.st)) break;
-        mbar_arrive_expect_tx(&full[s], CH * kBox);
-        for (int kk = 0; kk < S; ++kk)
-          for (int c = 0; c < CH; ++c)
-            tma_load_4d(&tm_k, &full[s], smem + L::K + s * CH * kBox + (kk * CH + c) * (R * 128),
-                        c * 64, g, j * kTile + S - 1 - kk, b);
-        issued = j + 1;
+      for (int t = 0; t < total; ++t) {
+        const int st = t % kStages;
+        if (t >= kStages && !mbar_wait(&empty[st], ((t / kStages) - 1) & 1, a.st)) break;
+        const int gi = t / NCHUNK, kk = (t % NCHUNK) / CH, c = t % CH;
+        mbar_arrive_expect_tx(&full[st], L::KC_BYTES);
+        for (int q4 = 0; q4 < 4; ++q4)
+          tma_load_4d(&tm_k, &full[st], smem + L::KC + st * L::KC_BYTES + q4 * 32 * 128, c * 64, g,
+                      (gi * kGroup + 2 * q4) * kTile + S - 1 - kk, b);
+        issued = t + 1;
       }
       mbar_drain(qbar, 0);
-      for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
-        mbar_drain(&full[j & 1], (j >> 1) & 1);
+      for (int t = issued - kStages < 0 ? 0 : issued - kStages; t < issued; ++t)
+        mbar_drain(&full[t % kStages], (t / kStages) & 1);
     }
-  } else if (warp < a.hc) {
-    // ------------------------------------------------------------ one query head
-    const int mi = lane >> 3, rr = lane & 7;     // ldmatrix: matrix, row within it
-    const int gq = lane >> 2, tq = lane & 3;     // mma fragment: row group, column pair
-    const uint32_t qbase = smem_u32(smem + L::Q + warp * CH * kBox);
-    const int ra = ((mi & 1) << 3) + rr;         // A: strided row of this lane's matrix row
-    const int cb = ((mi >> 1) << 3) + rr;        // B: strided column (two n-tiles of 8)
-    float* my_lse = lse + warp * a.nb;
-    bool ok = mbar_wait(qbar, 0, a.st);
-    for (int j = 0; ok && j <= i; ++j) {
-      const int s = j & 1;
-      if (!mbar_wait(&full[s], (j >> 1) & 1, a.st)) { ok = false; break; }
-      const uint32_t kbase = smem_u32(smem + L::K + s * CH * kBox);
-      // Two partial sums per n-tile (even / odd channel steps) halve the
-      // dependent MMA chains.
-      float acc[2][2][4] = {};
-#pragma unroll 1
-      for (int kk = 0; kk < S; ++kk) {
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // D[128 keys x 64 query rows] = Kc[128 x 8d] Q[64 x 8d]^T per group of 8 key
+    // blocks, double-buffered in TMEM columns [64 s, 64 s + 64): row = TMEM lane
+    // = strided key position, column 16 h + r = strided row r of head h.
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(kGroup * 16, L::QROWS, false, false);
+      const uint32_t qbase = smem_u32(smem + L::Q);
+      bool mok = mbar_wait(qbar, 0, a.st);
+      for (int gi = 0; mok && gi < ngroups; ++gi) {
+        const int gb = gi & 1;
+        if (gi >= 2 && !mbar_wait(&dfree[gb], ((gi >> 1) - 1) & 1, a.st)) { mok = false; break; }
+        for (int u = 0; u < NCHUNK; ++u) {
+          const int t = gi * NCHUNK + u, st = t % kStages;
+          if (!mbar_wait(&full[st], (t / kStages) & 1, a.st)) { mok = false; break; }
+          tc_fence_after();
+          const uint32_t kc = smem_u32(smem + L::KC + st * L::KC_BYTES);
+          const uint32_t qc = qbase + u * (L::QROWS * 128);   // u = kk * CH + c
 #pragma unroll
-        for (int dc = 0; dc < D / 16; ++dc) {
-          uint32_t af[4], b00, b01, b10, b11;
-          ldmatrix_x4(swz<R, CH>(qbase, kk, ra, dc * 2 + (mi >> 1)), af[0], af[1], af[2], af[3]);
-          ldmatrix_x4(swz<R, CH>(kbase, kk, cb, dc * 2 + (mi & 1)), b00, b01, b10, b11);
-          mma_bf16_16816(acc[0][dc & 1], af, b00, b01);
-          mma_bf16_16816(acc[1][dc & 1], af, b10, b11);
+          for (int k16 = 0; k16 < 4; ++k16)
+            umma_bf16_ss(tmem + gb * 64,
+                         umma_smem_desc(kc + k16 * 32, 16, 1024, kSwizzle128B),
+                         umma_smem_desc(qc + k16 * 32, 16, 1024, kSwizzle128B), idesc,
+                         (u | k16) != 0);
+          umma_commit(&empty[st]);
         }
+        if (!mok) break;
+        umma_commit(&dfull[gb]);
       }
+      // Every MMA issued by this thread completes before TMEM is released.
+      umma_commit(drain);
+      mbar_drain(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue: one lane quarter
+    // Warp w reads TMEM lanes 32 q .. 32 q + 31 (q = w % 4): key blocks 2q + (lane >> 4)
+    // of the group, strided key column lane & 15; 64 columns = 4 heads x 16 rows.
+    const int q = warp & 3;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const int half = lane >> 4, cc = lane & 15;
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int gb = gi & 1;
+      if (!mbar_wait(&dfull[gb], (gi >> 1) & 1, a.st)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t v[2][32];
+      tmem_ld32(tl + gb * 64, v[0]);
+      tmem_ld32(tl + gb * 64 + 32, v[1]);
+      tmem_wait_ld();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      // Block log-sum-exp (log2 domain) over the valid strided pairs c <= r.
-      float z[8];
-      float m = -INFINITY;
+      if (lane == 0) mbar_arrive(&dfree[gb]);
+      const int j = gi * kGroup + 2 * q + half;   // this lane's key block
+      const int cg = j * R + cc;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int h = 0; h < kMaxHeads; ++h) {
+        float z[16];
+        float m = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = gq + (e >> 1) * 8, c = nt * 8 + 2 * tq + (e & 1);
-          const int rg = i * R + r, cg = j * R + c;
-          const bool valid = cg <= rg && rg < a.nr && cg < a.nr;
-          const float v = valid ? (acc[nt][0][e] + acc[nt][1][e]) * a.scale_log2 : -INFINITY;
-          z[nt * 4 + e] = v;
-          m = fmaxf(m, v);
+        for (int r = 0; r < 16; ++r) {
+          const int rg = i * R + r;
+          const bool valid = j <= i && cg <= rg && rg < a.nr && cg < a.nr;
+          z[r] = valid ? __uint_as_float(v[h >> 1][(h & 1) * 16 + r]) * a.scale_log2 : -INFINITY;
+          m = fmaxf(m, z[r]);
+        }
+        // over the 16 lanes of this key block (xor within a half-warp)
+#pragma unroll
+        for (int o = 8; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float sum = 0.f;
+        if (m != -INFINITY) {
+#pragma unroll
+          for (int r = 0; r < 16; ++r) sum += ex2(z[r] - m);
         }
 #pragma unroll
-      for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      float sum = 0.f;
-      if (m != -INFINITY) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sum += ex2(z[e] - m);
+        for (int o = 8; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (cc == 0 && j <= i) lse[h * a.nb + j] = m == -INFINITY ? -INFINITY : m + __log2f(sum);
       }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) my_lse[j] = m == -INFINITY ? -INFINITY : m + __log2f(sum);
     }
-    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp >= 2) {
     // This head's shares: P_h[j] = 2^(lse_j - lse_total), written over lse.
+    float* my_lse = lse + (warp & 3) * a.nb;
     float mx = -INFINITY;
     for (int j = lane; j <= i; j += 32) mx = fmaxf(mx, my_lse[j]);
 #pragma unroll
@@ -208,10 +265,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   // The chunk's heads summed in a fixed order.
   float* out = a.partial + (static_cast<size_t>((b * a.Hkv + g) * nchunk + hc) * a.nb + i) * a.nb;
   for (int j = threadIdx.x; j <= i; j += blockDim.x) {
-    float s = 0.f;
-    for (int w = 0; w < a.hc; ++w) s += lse[w * a.nb + j];
-    out[j] = s;
+    float sacc = 0.f;
+    for (int w = 0; w < a.hc; ++w) sacc += lse[w * a.nb + j];
+    out[j] = sacc;
   }
+  if (warp == 1) tmem_dealloc(tmem, 128);
 }
 
 __global__ void __launch_bounds__(kSelectThreads)
