@@ -26,8 +26,8 @@
 //     head's rows being the first 16 lanes of its TMEM quarter) reduce each
 //     tile to the block's log-sum-exp while the next block's MMAs run, and
 //     at the end each head's shares are summed over the chunk into a
-//     per-chunk partial row.  Bound: the K tiles' stream from L2 (the heads
-//     of a kv group share them through the CTA).
+//     per-chunk partial row.  Bound: the K chunks' stream from L2 (each key
+//     block once per query block and chunk of heads; about 7 TB/s at T 32768).
 //   block_select_kernel: one CTA per query block: the partial rows summed in
 //     a fixed order, a bitonic sort of the candidates (score descending, block
 //     ascending) and one thread's sequential fp32 running sum decide the kept
