@@ -44,6 +44,10 @@ CASES = [  # B, T, Hq, Hkv, d, stride, tau, sink
     (1, 128, 2, 2, 64, 8, 0.5, 0),       # a single block
     (1, 3000, 5, 1, 64, 8, 0.9, 1),      # 5 heads per kv head: one per CTA
     (1, 2049, 4, 1, 128, 8, 0.7, 1),     # one token past a block boundary
+    (1, 1, 4, 1, 128, 8, 0.9, 1),        # a single token
+    (3, 130, 2, 1, 64, 8, 0.9, 0),       # two blocks, the second two tokens long; 2 heads per CTA
+    (1, 1100, 1, 1, 64, 8, 0.6, 20),     # sink beyond the block count: every block forced
+    (1, 4500, 8, 2, 128, 8, 0.99, 1),    # 9 key-block groups of 8 at the last query block
 ]
 
 
