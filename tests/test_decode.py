@@ -1,4 +1,4 @@
-"""Split-KV decode attention against the fp64 oracle (FA and SA per layer)."""
+"""Split-KV decode attention against the fp64 oracle (FA and SA per layer; GQA group sizes 1 to 8)."""
 import math
 
 import numpy as np
