@@ -160,6 +160,30 @@ def test_qwen3_4b_layer_prefill_sampled_rows(ctx, mode):
             assert np.abs(synth.bf16_bits_to_f32(o[0, r, h]) - target).max() < 0.1
 
 
+@pytest.mark.parametrize("mode", [1, 0])
+def test_batch_of_two_chunked_unit_order(ctx, mode):
+    """B 2, ragged T 20000, Hkv 8: the K/V of one kv group take 10 MB, so units run per
+    sequence in chunks of 4 kv groups (of 8); sampled rows of both sequences and every
+    head against the oracle, FA and SA (block 128, sink 1, window 16)."""
+    B, T, Hq, Hkv, d = 2, 20000, 16, 8, 128
+    q, k, v = synth.attention_inputs(B, T, Hq, Hkv, d, seed=4242)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = _run(ctx, q, k, v, scale, mode, 128, 1, 16)
+    r = synth.rng(4243)
+    rows = []
+    for b in range(B):
+        for h in range(Hq):
+            ts = set(int(x) for x in r.integers(0, T, 12)) | {0, 127, 128, T - 129, T - 1}
+            rows += [(b, h, t) for t in sorted(ts)]
+    rows = np.array(rows, np.int32)
+    nb = (T + 127) // 128
+    m = oracle.streaming_mask(nb, nb, 1, 16) if mode == 0 else None
+    ro, rl = oracle.attn_prefill(q, k, v, scale, block_mask=m, block=128, rows=rows)
+    got = o[rows[:, 0], rows[:, 2], rows[:, 1]]
+    assert_close_attn(got, ro, f"B 2 T 20000 mode {mode}")
+    assert_close_lse(lse[rows[:, 0], rows[:, 1], rows[:, 2]], rl, "lse")
+
+
 def _random_causal_block_mask(nb, keep, seed):
     r = np.random.default_rng(seed)
     m = (r.random((nb, nb)) < keep).astype(np.uint8)
