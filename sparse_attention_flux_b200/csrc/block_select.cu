@@ -15,19 +15,19 @@
 // Two kernels:
 //   block_score_kernel: one CTA per (sequence, kv head, chunk of up to four
 //     query heads, query block i), query blocks longest first.  TMA brings
-//     the chunk's Q once and the K tile of every key block j <= i through a
-//     2-stage ring, each as 8 strided boxes (traversal stride 8): box kk holds
-//     the 16 rows kk, kk + 8, ... of Q (for K: 7-kk, 15-kk, ...), so the
-//     strided positions are consecutive rows and the antidiagonal pairing is
-//     the choice of box.  Q is the resident A operand of one tcgen05 MMA chain
-//     per key block: M 64 = four heads x 16 strided positions, N 16 strided
-//     key positions, K = 8 d (64 MMAs of K 16 at d 128), accumulated in a
-//     double-buffered TMEM tile; four epilogue warps (one per head, the
-//     head's rows being the first 16 lanes of its TMEM quarter) reduce each
-//     tile to the block's log-sum-exp while the next block's MMAs run, and
-//     at the end each head's shares are summed over the chunk into a
-//     per-chunk partial row.  Bound: the K chunks' stream from L2 (each key
-//     block once per query block and chunk of heads; about 7 TB/s at T 32768).
+//     the chunk's Q once as strided boxes (traversal stride 8: box kk holds
+//     the 16 rows kk, kk + 8, ... of block i), resident in shared memory as
+//     the N = 64 operand (four heads x 16 strided rows).  The keys are the
+//     M = 128 operand: 8 key blocks x 16 strided positions, boxes of rows
+//     7-kk, 15-kk, ... so the antidiagonal pairing is the choice of box,
+//     streamed as 16 KB chunks (one offset kk, 64 channels) through a 4-stage
+//     ring; K = 8 d per tile.  The 128-lane x 64-column accumulator is
+//     double-buffered in TMEM; four epilogue warps, one per lane quarter (two
+//     key blocks each), reduce it to per-(head, key block) log-sum-exps while
+//     the next tile's MMAs run, and at the end each head's shares are summed
+//     over the chunk into a per-chunk partial row.  Bound: the K chunks'
+//     stream from L2 (each key block once per query block and chunk of heads;
+//     about 7 TB/s at T 32768).
 //   block_select_kernel: one CTA per query block: the partial rows summed in
 //     a fixed order, a bitonic sort of the candidates (score descending, block
 //     ascending) and one thread's sequential fp32 running sum decide the kept
