@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
             L.oracle_attn_decode.argtypes = [_u16p, _u16p, _u16p, i, _i32p, i, i, i, i, i, i, i,
                                              i, d, _f64p, _vp]
             L.oracle_block_scores.argtypes = [_u16p, _u16p, i, i, i, i, i, i, i, d, _f64p]
+            L.oracle_block_scores_rows.argtypes = [_u16p, _u16p, i, i, i, i, i, i, i, d,
+                                                   _i32p, i, _f64p]
             L.oracle_select_blocks.argtypes = [_f32p, i, f, i, _u8p]
             _lib = L
     return _lib
@@ -260,6 +262,24 @@ def block_scores(q, k, block: int, stride: int, scale: float) -> np.ndarray:
     P = np.zeros((nb, nb), np.float64)
     _check(lib().oracle_block_scores(q, k, B, T, Hq, Hkv, d, block, stride, scale, P),
            "block_scores")
+    return P
+
+
+def block_scores_rows(q, k, block: int, stride: int, scale: float, rows) -> np.ndarray:
+    """The rows of block_scores for the query blocks listed in ``rows`` only:
+    fp64 [len(rows), nb], row n = query block rows[n] (a query block's row
+    depends on its own queries alone).  Parity unpinned against the pages."""
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    rows = np.ascontiguousarray(rows, np.int32)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    nr = (T + stride - 1) // stride
+    R = block // stride
+    nb = (nr + R - 1) // R
+    P = np.zeros((len(rows), nb), np.float64)
+    _check(lib().oracle_block_scores_rows(q, k, B, T, Hq, Hkv, d, block, stride, scale, rows,
+                                          len(rows), P), "block_scores_rows")
     return P
 
 

@@ -421,16 +421,22 @@ int oracle_attn_decode(const uint16_t* q, const uint16_t* k_cache, const uint16_
  *   layer score  P[i][j] = mean over (b, h) of P_h[i][j].
  * Parity unpinned against the pages (they print no algorithm); these
  * functions are pinned to brute force, closed forms and invariants of the
- * definition above.
+ * definition above.  oracle_block_scores_rows computes the rows of the
+ * listed query blocks only (P [nrows][nb], row n = query block rows[n]):
+ * each row depends on its own block's queries alone, so large layers are
+ * checked on sampled rows.
  */
-int oracle_block_scores(const uint16_t* q, const uint16_t* k, int B, int T, int Hq, int Hkv,
-                        int d, int block, int stride, double scale, double* P) {
+int oracle_block_scores_rows(const uint16_t* q, const uint16_t* k, int B, int T, int Hq,
+                             int Hkv, int d, int block, int stride, double scale,
+                             const int* rows, int nrows, double* P) {
     if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || d < 1 || stride < 1 ||
-        block < stride || block % stride) return -1;
+        block < stride || block % stride || nrows < 1 || !rows) return -1;
     const int G = Hq / Hkv, S = stride, R = block / S;
     const int nr = (T + S - 1) / S, nb = (nr + R - 1) / R;
+    for (int n = 0; n < nrows; ++n)
+        if (rows[n] < 0 || rows[n] >= nb) return -1;
     const int nbh = B * Hq;
-    double* Ph = (double*)calloc((size_t)nbh * nb * nb, sizeof(double));
+    double* Ph = (double*)calloc((size_t)nbh * nrows * nb, sizeof(double));
     if (!Ph) return -1;
     int bad = 0;
 #pragma omp parallel
@@ -439,13 +445,13 @@ int oracle_block_scores(const uint16_t* q, const uint16_t* k, int B, int T, int 
         double* ks = (double*)malloc(sizeof(double) * (size_t)S * d);       /* one strided col */
         double* z = (double*)malloc(sizeof(double) * (size_t)R * nr);
 #pragma omp for schedule(dynamic, 1)
-        for (long long w = 0; w < (long long)nbh * nb; ++w) {
+        for (long long w = 0; w < (long long)nbh * nrows; ++w) {
             if (!qs || !ks || !z) {
 #pragma omp atomic write
                 bad = 1;
                 continue;
             }
-            const int bh = (int)(w / nb), i = (int)(w % nb);
+            const int bh = (int)(w / nrows), n = (int)(w % nrows), i = rows[n];
             const int b = bh / Hq, h = bh % Hq, g = h / G;
             const int r0 = i * R, r1 = r0 + R < nr ? r0 + R : nr;
             /* the query rows of block i, widened (zero past T) */
@@ -479,7 +485,7 @@ int oracle_block_scores(const uint16_t* q, const uint16_t* k, int B, int T, int 
                 }
             }
             /* block masses relative to exp(zmax), then their shares */
-            double* row = Ph + ((size_t)bh * nb + i) * nb;
+            double* row = Ph + ((size_t)bh * nrows + n) * nb;
             double tot = 0.0;
             for (int j = 0; j <= i; ++j) {
                 double e = 0.0;
@@ -497,14 +503,28 @@ int oracle_block_scores(const uint16_t* q, const uint16_t* k, int B, int T, int 
     }
     if (!bad) {
         /* mean over (b, h), summed in a fixed order */
-        for (size_t e = 0; e < (size_t)nb * nb; ++e) {
+        for (size_t e = 0; e < (size_t)nrows * nb; ++e) {
             double s = 0.0;
-            for (int bh = 0; bh < nbh; ++bh) s += Ph[(size_t)bh * nb * nb + e];
+            for (int bh = 0; bh < nbh; ++bh) s += Ph[(size_t)bh * nrows * nb + e];
             P[e] = s / nbh;
         }
     }
     free(Ph);
     return bad ? -1 : 0;
+}
+
+/* All query blocks: P [nb][nb]. */
+int oracle_block_scores(const uint16_t* q, const uint16_t* k, int B, int T, int Hq, int Hkv,
+                        int d, int block, int stride, double scale, double* P) {
+    if (T < 1 || stride < 1 || block < stride || block % stride) return -1;
+    const int R = block / stride, nr = (T + stride - 1) / stride, nb = (nr + R - 1) / R;
+    int* rows = (int*)malloc(sizeof(int) * (size_t)nb);
+    if (!rows) return -1;
+    for (int i = 0; i < nb; ++i) rows[i] = i;
+    const int rc = oracle_block_scores_rows(q, k, B, T, Hq, Hkv, d, block, stride, scale, rows,
+                                            nb, P);
+    free(rows);
+    return rc;
 }
 
 /*

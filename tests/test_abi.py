@@ -111,6 +111,8 @@ def test_select_blocks_host_checks_need_no_gpu(lib):
         flux.FLUX_ERR_UNSUPPORTED
     assert f(ctx, P, P, 1, 200000, 2, 1, 64, 128, 8, 0.125, 0.9, 0, M, None, None) == \
         flux.FLUX_ERR_UNSUPPORTED
+    assert f(ctx, P, P, 1, 131073, 2, 1, 64, 128, 8, 0.125, 0.9, 0, M, None, None) == \
+        flux.FLUX_ERR_UNSUPPORTED   # 1025 blocks: one past the largest layer
     assert f(ctx, P, P, 1, 256, 3, 2, 64, 128, 8, 0.125, 0.9, 0, M, None, None) == \
         flux.FLUX_ERR_UNSUPPORTED
     assert f(ctx, P, P, 1, 256, 2, 1, 64, 128, 8, float("nan"), 0.9, 0, M, None, None) == \

@@ -109,3 +109,54 @@ def test_deterministic(ctx):
     m1, s1 = _select(ctx, q, k, 8, 0.9, 1)
     m2, s2 = _select(ctx, q, k, 8, 0.9, 1)
     assert np.array_equal(m1, m2) and np.array_equal(s1, s2)
+
+
+def _sampled_rows_check(score, mask, q, k, d, rows, tau, sink, what):
+    """Sampled score rows against the oracle, then properties of the whole GPU matrix:
+    rows sum to 1, nothing above the diagonal, and the mask is the oracle's selection
+    on the GPU's fp32 scores, bit for bit."""
+    nb = score.shape[0]
+    P = oracle.block_scores_rows(q, k, 128, 8, 1 / math.sqrt(d), rows)
+    for n, i in enumerate(rows):
+        err = np.abs(score[i, :i + 1].astype(np.float64) - P[n, :i + 1])
+        assert err.max() <= 5e-5 + 1e-3 * P[n, :i + 1].max(), f"{what}: row {i} error {err.max()}"
+    upper = np.triu(np.ones((nb, nb), bool), 1)
+    assert np.all(score[upper] == 0) and np.all(mask[upper] == 0)
+    np.testing.assert_allclose(score.astype(np.float64).sum(axis=1), 1.0, atol=1e-4)
+    np.testing.assert_array_equal(mask, oracle.select_blocks(score, tau, sink), err_msg=what)
+
+
+def test_qwen3_4b_layer_sampled_rows(ctx):
+    """The bench's layer: B 1, T 32768, Hq 32, Hkv 8, d 128 with planted needles;
+    stride 8, tau 0.9, sink 1.  Sampled query blocks (first, second, last, every needle
+    row's block, and seeded others) against the oracle; the whole mask bit-exact on the
+    GPU's scores; and the selected mask keeps more of the needles' key blocks than the
+    sink + window mask."""
+    B, T, Hq, Hkv, d, tau, sink = 1, 32768, 32, 8, 128, 0.9, 1
+    seed = synth.seed_for(1)
+    q, k, _ = synth.attention_inputs(B, T, Hq, Hkv, d, seed)
+    needles = synth.plant_needles_np(q, k, seed)
+    mask, score = _select(ctx, q, k, 8, tau, sink)
+    nb = T // 128
+    r = synth.rng(seed + 9)
+    rows = sorted({0, 1, nb - 1} | {rr // 128 for (_, rr, _) in needles}
+                  | set(int(x) for x in r.integers(0, nb, 6)))
+    _sampled_rows_check(score, mask, q, k, d, rows, tau, sink, "T 32768")
+    stream = oracle.streaming_mask(nb, nb, sink, 16)
+    hit_sel = hit_stream = 0
+    for (_h, rr, pos) in needles:
+        for j in set(int(p) // 128 for p in pos):
+            hit_sel += int(mask[rr // 128, j])
+            hit_stream += int(stream[rr // 128, j])
+    assert hit_sel > hit_stream
+
+
+def test_largest_supported_layer(ctx):
+    """T 131072 = 1024 key blocks, the largest the selector takes (the shared-memory
+    log-sum-exp row and the sort are sized for it): sampled rows against the oracle and
+    the whole mask bit-exact (one token more is refused on the host: test_abi)."""
+    B, T, Hq, Hkv, d, tau, sink = 1, 131072, 4, 1, 128, 0.9, 1
+    q, k, _ = synth.attention_inputs(B, T, Hq, Hkv, d, seed=777)
+    mask, score = _select(ctx, q, k, 8, tau, sink)
+    assert score.shape == (1024, 1024)
+    _sampled_rows_check(score, mask, q, k, d, [0, 7, 8, 513, 1016, 1023], tau, sink, "T 131072")

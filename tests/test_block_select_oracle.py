@@ -169,3 +169,26 @@ def test_selection_matches_restated_rule(seed):
     tau = float(rng.choice([0.5, 0.8, 0.9, 0.95]))
     sink = int(rng.integers(0, 3))
     np.testing.assert_array_equal(oracle.select_blocks(P, tau, sink), _select_reference(P, tau, sink))
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,d,rows", [
+    (1000, 4, 2, 64, [7, 0, 3]),        # unsorted, first and last blocks
+    (777, 3, 1, 32, [6, 6, 2]),         # ragged T, a repeated block
+    (300, 2, 2, 16, [1]),
+])
+def test_sampled_rows_equal_full_matrix(T, Hq, Hkv, d, rows):
+    # Each query block's row depends on its own queries only: the sampled rows are the
+    # full matrix's rows, bit for bit.
+    q, k, _ = synth.attention_inputs(2, T, Hq, Hkv, d, seed=T + d)
+    P = oracle.block_scores(q, k, 128, 8, 1 / np.sqrt(d))
+    Pr = oracle.block_scores_rows(q, k, 128, 8, 1 / np.sqrt(d), rows)
+    assert Pr.shape == (len(rows), P.shape[0])
+    np.testing.assert_array_equal(Pr, P[rows])
+
+
+def test_sampled_rows_reject_out_of_range():
+    q, k, _ = synth.attention_inputs(1, 256, 2, 1, 16, seed=1)
+    with pytest.raises(ValueError):
+        oracle.block_scores_rows(q, k, 128, 8, 0.25, [2])
+    with pytest.raises(ValueError):
+        oracle.block_scores_rows(q, k, 128, 8, 0.25, [-1])
