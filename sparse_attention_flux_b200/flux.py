@@ -234,6 +234,8 @@ class Context:
         _need(block_mask, torch.uint8, "block_mask", self.device)
         B, T, Hq, d = q.shape
         Hkv = k.shape[2]
+        if k.shape != (B, T, Hkv, d):
+            raise ValueError("q/k shapes are inconsistent")
         nb = (T + block - 1) // block
         if block_mask.numel() < nb * nb:
             raise ValueError("block_mask needs nb * nb entries")
@@ -314,10 +316,17 @@ class Context:
             _need(t, torch.bfloat16, n_, self.device)
         _need(head_mode, torch.uint8, "head_mode", self.device)
         _need(lse, torch.float32, "lse", self.device)
+        _need(row_ptr, torch.int32, "row_ptr", self.device)
+        _need(col, torch.int32, "col", self.device)
+        if row_ptr is None or col is None:
+            raise ValueError("row_ptr and col are required")
         B, T, Hq, d = q.shape
         Hkv = k.shape[2]
-        if head_mode.numel() < Hq or k.shape != (B, T, Hkv, d) or v.shape != k.shape:
+        if head_mode.numel() < Hq or k.shape != (B, T, Hkv, d) or v.shape != k.shape \
+                or o.shape != q.shape:
             raise ValueError("shapes are inconsistent")
+        if lse is not None and lse.numel() < B * Hq * T:
+            raise ValueError("lse too small")
         _check(lib().flux_attn_prefill_heads(self._h, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                              B, T, Hq, Hkv, d, _ptr(head_mode), _ptr(row_ptr),
                                              _ptr(col), row_ptr.numel() - 1, block, float(scale),
@@ -334,8 +343,11 @@ class Context:
         _need(lse, torch.float32, "lse", self.device)
         B, Hq, d = q.shape
         _, S_max, Hkv, _ = k_cache.shape
-        if head_mode.numel() < Hq or v_cache.shape != k_cache.shape:
+        if head_mode.numel() < Hq or k_cache.shape != (B, S_max, Hkv, d) \
+                or v_cache.shape != k_cache.shape or o.shape != q.shape or seqlens.numel() < B:
             raise ValueError("shapes are inconsistent")
+        if lse is not None and lse.numel() < B * Hq:
+            raise ValueError("lse too small")
         _check(lib().flux_attn_decode_heads(self._h, _ptr(q), _ptr(k_cache), _ptr(v_cache), S_max,
                                             _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, d,
                                             _ptr(head_mode), sink_blocks, window_blocks, block,
@@ -394,8 +406,11 @@ class Context:
         B, Hq, d = q.shape
         _, rows, Hkv, _ = k_cache.shape
         if k_cache.shape[0] != B or k_cache.shape[3] != d or v_cache.shape != k_cache.shape \
-                or o.shape != q.shape or k_new.numel() != B * Hkv * d or v_new.shape != k_new.shape:
+                or o.shape != q.shape or k_new.numel() != B * Hkv * d or v_new.shape != k_new.shape \
+                or seqlens.numel() < B:
             raise ValueError("q / k_new / cache / o shapes are inconsistent")
+        if lse is not None and lse.numel() < B * Hq:
+            raise ValueError("lse too small")
         _check(lib().flux_attn_decode_append(self._h, _ptr(q), _ptr(k_new), _ptr(v_new),
                                              _ptr(k_cache), _ptr(v_cache), rows, _ptr(seqlens),
                                              _ptr(o), _ptr(lse), B, Hq, Hkv, d, _ptr(layer_mode),
@@ -417,8 +432,11 @@ def attn_decode_noalloc(q, k_cache, v_cache, seqlens, o, scale: float, layer_mod
     _need(status, torch.int32, "status")
     B, Hq, d = q.shape
     _, S_max, Hkv, _ = k_cache.shape
-    if k_cache.shape != (B, S_max, Hkv, d) or v_cache.shape != k_cache.shape or o.shape != q.shape:
+    if k_cache.shape != (B, S_max, Hkv, d) or v_cache.shape != k_cache.shape or o.shape != q.shape \
+            or seqlens.numel() < B:
         raise ValueError("q/cache/o shapes are inconsistent")
+    if lse is not None and lse.numel() < B * Hq:
+        raise ValueError("lse too small")
     _check(lib().flux_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), S_max,
                                           _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv, d,
                                           _ptr(layer_mode), layer, sink_blocks, window_blocks,
