@@ -154,7 +154,8 @@ int flux_build_streaming_mask(int nqb, int nkb, int sink_blocks, int window_bloc
  *   block_mask [nb, nb] uint8 out; block_score [nb, nb] fp32 out (optional,
  *   zero above the diagonal).
  * Supported: d 64 or 128, block 128, stride 8, T <= 131072.  Uses
- * flux_select_blocks_workspace_bytes() bytes of the ctx workspace.
+ * flux_select_blocks_workspace_bytes() bytes of the ctx workspace (that query
+ * returns 0 for a shape this call does not support).
  * Errors: INVALID_ARG (null pointers, scale not finite and positive, tau
  * negative or not finite, sink_blocks < 0, misaligned q/k), UNSUPPORTED
  * (d, block, stride, T, Hq % Hkv), SHAPE (sizes, workspace too small). */

@@ -415,7 +415,9 @@ int flux_route(flux_ctx* c, const uint16_t* hidden, int T, int Hd, int n_pool, c
 }
 
 size_t flux_select_blocks_workspace_bytes(int B, int T, int Hq, int Hkv, int stride) {
-  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || stride != 8) return 0;
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || stride != 8 ||
+      (T + 127) / 128 > flux::kSelectMaxBlocks)
+    return 0;
   return flux::block_select_workspace_bytes(B, T, Hq, Hkv, stride);
 }
 

@@ -125,3 +125,5 @@ def test_select_blocks_host_checks_need_no_gpu(lib):
     nb = 32768 // 128
     assert lib.flux_select_blocks_workspace_bytes(1, 32768, 32, 8, 8) == 8 * nb * nb * 4
     assert lib.flux_select_blocks_workspace_bytes(1, 256, 3, 2, 8) == 0
+    assert lib.flux_select_blocks_workspace_bytes(1, 131073, 4, 1, 8) == 0   # above the largest
+    assert lib.flux_select_blocks_workspace_bytes(1, 131072, 4, 1, 8) == 1024 * 1024 * 4
