@@ -932,11 +932,7 @@ def run_flux(args, rank, world, dev_index):
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "qwen3-4b-layer-routed-prefill: B 1, T 32768, Hq 32, Hkv 8, d 128, "
-                               "needles; router 32768x2560 -> MLP 5120-512-2 (layer0 FA, layer1 SA); "
-                               "SA block 128, sink 1, window 16",
-                   "l2": "inputs larger than L2 (640 MB prefill, 17 GB decode KV); no flush",
-                   "parallelism": f"replicas x{world} (no exchange)"},
+        "config": bench_config(world),
         "roofline": {"bound": "tensor", "achieved": round(fa_tflops, 1), "peak": peak_t,
                      "unit": "TFLOP/s", "frac": round(fa_tflops / peak_t, 4),
                      "traffic": recorded_traffic("prefill_fa_T32768"),
@@ -975,47 +971,102 @@ def run_flux(args, rank, world, dev_index):
     return line
 
 
-def cpu_baseline(seconds_budget=15.0, threads=None):
-    """The oracle, as it stands, on a bounded sample of the same prefill workload
-    (all host cores, or `threads` of them)."""
-    import oracle
+def bench_config(world: int) -> dict:
+    """The workload both arms (this library and the oracle) report."""
+    return {"workload": "qwen3-4b-layer-routed-prefill: B 1, T 32768, Hq 32, Hkv 8, d 128, "
+                        "needles; router 32768x2560 -> MLP 5120-512-2 (layer0 FA, layer1 SA); "
+                        "SA block 128, sink 1, window 16",
+            "l2": "inputs larger than L2 (640 MB prefill, 17 GB decode KV); no flush",
+            "parallelism": f"replicas x{world} (no exchange)"}
+
+
+class OracleSample:
+    """The oracle, as it stands, on bounded samples of the bench's prefill layer:
+    uniformly drawn query rows, FA rows for half of a sample's time, then SA rows.
+    FLOPs are counted like the GPU's (4 d per visible pair)."""
+
+    def __init__(self):
+        import oracle
+        from sparse_attention_flux_b200 import synth
+        self.oracle = oracle
+        seed = synth.seed_for(1)
+        self.q, self.k, self.v = synth.attention_inputs(1, T, HQ, HKV, D, seed)
+        synth.plant_needles_np(self.q, self.k, seed)
+        self.scale = 1.0 / math.sqrt(D)
+        nb = T // BLOCK
+        self.mask = oracle.streaming_mask(nb, nb, SINK, WIN)
+        self.r = synth.rng(seed + 9)
+
+    def run(self, seconds):
+        """One bounded sample: (visible pairs, seconds taken, rows)."""
+        pairs, used, n_rows = 0, 0.0, 0
+        for sparse in (False, True):
+            t0 = time.perf_counter()
+            while time.perf_counter() - t0 < seconds / 2:
+                rows = np.stack([np.zeros(64, np.int32),
+                                 self.r.integers(0, HQ, 64).astype(np.int32),
+                                 self.r.integers(0, T, 64).astype(np.int32)], 1)
+                self.oracle.attn_prefill(self.q, self.k, self.v, self.scale,
+                                         block_mask=self.mask if sparse else None, block=BLOCK,
+                                         rows=rows)
+                for t in rows[:, 2]:
+                    if sparse:
+                        i = t // BLOCK
+                        pairs += sum(min(BLOCK, t + 1 - j * BLOCK) for j in range(i + 1)
+                                     if (j < SINK or j >= i - WIN + 1))
+                    else:
+                        pairs += t + 1
+                n_rows += 64
+            used += time.perf_counter() - t0
+        return pairs, used, n_rows
+
+
+def cpu_baseline(seconds_budget=15.0, threads=None, sampler=None):
+    """The oracle on one bounded sample of the same prefill workload (all host cores,
+    or `threads` of them)."""
+    sampler = sampler or OracleSample()
+    oracle = sampler.oracle
     if threads is not None:
         all_threads = oracle.num_threads()
         oracle.set_num_threads(threads)
-    from sparse_attention_flux_b200 import synth
-    seed = synth.seed_for(1)
-    q, k, v = synth.attention_inputs(1, T, HQ, HKV, D, seed)
-    synth.plant_needles_np(q, k, seed)
-    scale = 1.0 / math.sqrt(D)
-    nb = T // BLOCK
-    m = oracle.streaming_mask(nb, nb, SINK, WIN)
-    r = synth.rng(seed + 9)
-    # Sample rows uniformly; time FA rows until the budget is half spent, then SA rows.
-    done_pairs, t_used, n_rows = 0, 0.0, 0
-    for sparse in (False, True):
-        budget = seconds_budget / 2
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < budget:
-            rows = np.stack([np.zeros(64, np.int32), r.integers(0, HQ, 64).astype(np.int32),
-                             r.integers(0, T, 64).astype(np.int32)], 1)
-            oracle.attn_prefill(q, k, v, scale, block_mask=m if sparse else None, block=BLOCK,
-                                rows=rows)
-            for t in rows[:, 2]:
-                if sparse:
-                    i = t // BLOCK
-                    done_pairs += sum(min(BLOCK, t + 1 - j * BLOCK) for j in range(i + 1)
-                                      if (j < SINK or j >= i - WIN + 1))
-                else:
-                    done_pairs += t + 1
-            n_rows += 64
-        t_used += time.perf_counter() - t0
-    tflops = 4.0 * D * done_pairs / t_used / 1e12
+    pairs, used, n_rows = sampler.run(seconds_budget)
     cores = oracle.num_threads()
     if threads is not None:
         oracle.set_num_threads(all_threads)
-    return {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+    return {"value": 4.0 * D * pairs / used / 1e12, "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
             "sample": f"{n_rows} uniformly sampled query rows (half FA, half SA) of the T=32768 "
-                      f"layer, {t_used:.1f} s; FLOPs counted like the GPU's (4 d per visible pair)"}
+                      f"layer, {used:.1f} s; FLOPs counted like the GPU's (4 d per visible pair)"}
+
+
+def run_reference(args, world):
+    """The reference arm: the oracle on the host cores, W untimed and K timed steps,
+    each step a bounded sample of the bench's workload (sized so that the whole run
+    takes about 150 s), value = FLOPs of all timed steps / their time."""
+    sampler = OracleSample()                     # inputs prepared before timing, as on the GPU
+    per_step = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        sampler.run(per_step)
+    pairs = rows = 0
+    used = 0.0
+    for _ in range(args.steps):
+        p, u, n = sampler.run(per_step)
+        pairs, used, rows = pairs + p, used + u, rows + n
+    value = 4.0 * D * pairs / used / 1e12
+    sample = (f"{args.steps} steps of {per_step:.2f} s each ({args.warmup} more untimed): "
+              f"{rows} uniformly sampled query rows of the T=32768 layer (half of each step FA "
+              f"rows, half SA rows); FLOPs counted like the GPU's (4 d per visible pair)")
+    return {"metric": "routed-attn prefill TFLOP/s & decode KV GB/s at 1 B200; % of roofline",
+            "impl": "reference", "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": used / max(1, args.steps) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": bench_config(world),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s",
+                             "cores": sampler.oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
 
 
 def main():
@@ -1041,19 +1092,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        base = cpu_baseline(args.cpu_seconds)
-        per_step_s = args.cpu_seconds
-        line = {"metric": "routed-attn prefill TFLOP/s & decode KV GB/s at 1 B200; % of roofline",
-                "impl": "reference", "value": base["value"], "unit": "TFLOP/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": per_step_s * 1e3, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "qwen3-4b-layer-routed-prefill: B 1, T 32768, Hq 32, Hkv 8, "
-                                       "d 128 (sampled rows)"},
-                "cpu_baseline": base,
-                "e2e": {"value": base["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line))
+        print(json.dumps(run_reference(args, world)))
         return
 
     import torch
@@ -1066,8 +1105,9 @@ def main():
     line = run_flux(args, rank, world, local)
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
-            one = cpu_baseline(4.0, threads=1)
+            sampler = OracleSample()
+            line["cpu_baseline"] = cpu_baseline(args.cpu_seconds, sampler=sampler)
+            one = cpu_baseline(4.0, threads=1, sampler=sampler)
             line["cpu_baseline"]["single_thread"] = {"value": one["value"], "cores": 1,
                                                      "sample": one["sample"]}
         print(json.dumps(line))

@@ -62,3 +62,29 @@ def test_flop_and_byte_counts_match_closed_forms():
     assert bench.pairs_sa(256, 64, 1, 2) == 5 * full + 4 * diag
     assert bench.sa_decode_tokens(131072, 128, 1, 16) == 128 + 16 * 128
     assert bench.sa_decode_tokens(131072 + 5, 128, 1, 16) == 128 + 15 * 128 + 5
+
+
+def test_reference_arm_steps_and_config(monkeypatch):
+    """The reference arm runs W untimed and K timed bounded samples and reports the same
+    workload config as the library's arm; value = FLOPs of the timed steps / their time."""
+    calls = []
+
+    class FakeSample:
+        class oracle:
+            @staticmethod
+            def num_threads():
+                return 3
+
+        def run(self, seconds):
+            calls.append(seconds)
+            return 1000, 0.5, 64          # visible pairs, seconds, rows
+
+    monkeypatch.setattr(bench, "OracleSample", FakeSample)
+    args = type("A", (), {"steps": 4, "warmup": 3, "gpus": 1})()
+    line = bench.run_reference(args, 1)
+    assert len(calls) == 7 and all(0.5 <= c <= 4.0 for c in calls)
+    assert line["impl"] == "reference" and line["config"] == bench.bench_config(1)
+    assert line["value"] == pytest.approx(4.0 * bench.D * 4000 / 2.0 / 1e12)
+    assert line["ms_per_step"] == pytest.approx(500.0)
+    assert line["cpu_baseline"]["cores"] == 3 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
