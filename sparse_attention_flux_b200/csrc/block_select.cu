@@ -56,6 +56,9 @@ struct ScoreArgs {
 
 constexpr int kGroup = 8;                  // key blocks per MMA tile: M = 128 strided keys
 constexpr int kStages = 4;                 // K chunk ring
+// The barrier area (16 slots of 8 bytes) holds full and empty per stage, dfull[2],
+// dfree[2], qbar, drain and then the TMEM address slot.
+static_assert(2 * kStages + 6 + 1 <= 16, "barrier area too small for the ring");
 
 template <int D>
 struct ScoreSmem {
