@@ -347,12 +347,14 @@ int flux_attn_decode_heads(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_c
  *   partials within the 32 MiB (nsplit as flux_decode_workspace_bytes plans
  *   it; e.g. B 16, Hq 32, d 128 at 131072 tokens takes 4 splits, 1.1 MiB).  Larger shapes
  *   return FLUX_ERR_SHAPE before any device work.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.  Every call clears the error word and the
- *   tickets it uses on `stream`, then reuses the same array: calls that
- *   overlap on the GPU (on different streams or host threads) race and must
- *   be serialised by the caller. */
+ *   Every call looks up the array's device address on the current device
+ *   (cudaGetSymbolAddress, a host query that allocates nothing), so the entry
+ *   point stays valid after cudaDeviceReset.  The first call on a device may
+ *   load the library's device code there; make that first call before any
+ *   stream capture.  Every call clears the error word and the tickets it uses
+ *   on `stream`, then reuses the same array: calls that overlap on the GPU (on
+ *   different streams or host threads) race and must be serialised by the
+ *   caller. */
 int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cache, const uint16_t* v_cache,
                              int S_max, const int32_t* seqlens, uint16_t* o, float* lse,
                              int B, int Hq, int Hkv, int d,

@@ -607,8 +607,12 @@ int flux_attn_decode_append(flux_ctx* c, const uint16_t* q, const uint16_t* k_ne
 // cudaMalloc's implicit synchronisation).  Its scratch is the static array
 // below, which every device that loads libflux.so holds until the process
 // exits.  Host code must not pass the array's name to a kernel -- on the host
-// it is only a stand-in symbol -- so each device's address is looked up once,
-// with that device current, and cached.
+// it is only a stand-in symbol -- so every call looks up the array's device
+// address on the current device.  The lookup is a host query that allocates
+// nothing; doing it per call (rather than caching the address) keeps the entry
+// point valid after cudaDeviceReset, which unloads the module and gives the
+// array a new address when the next call loads it again.  Only the SM count is
+// cached per device.
 namespace {
 
 constexpr size_t kNoAllocBytes = size_t(32) << 20;        // 32 MiB
@@ -619,35 +623,29 @@ constexpr size_t kNoAllocPartOff = kNoAllocTicketOff + kNoAllocMaxGroups * sizeo
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-struct NoAllocDevice {
-  bool ready;
-  char* base;   // device address of g_noalloc_scratch on this device
-  int num_sms;
-};
 constexpr int kNoAllocMaxDevices = 64;
-NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+int g_noalloc_sms[kNoAllocMaxDevices];   // 0 = not yet queried
 std::mutex g_noalloc_mu;
 
-int noalloc_setup(NoAllocDevice** out) {
+// The scratch array's device address and the SM count of the current device.
+int noalloc_setup(char** base, int* num_sms) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: cudaGetDevice");
   if (dev < 0 || dev >= kNoAllocMaxDevices)
     return fail(FLUX_ERR_UNSUPPORTED, "flux_attn_decode_noalloc: device %d out of range", dev);
+  void* ptr = nullptr;
+  if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess)
+    return cuda_fail(e, "flux_attn_decode_noalloc: cudaGetSymbolAddress");
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  NoAllocDevice& d = g_noalloc_dev[dev];
-  if (!d.ready) {
-    void* ptr = nullptr;
-    if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess)
-      return cuda_fail(e, "flux_attn_decode_noalloc: cudaGetSymbolAddress");
+  if (g_noalloc_sms[dev] == 0) {
     int sms = 0;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
       return cuda_fail(e, "flux_attn_decode_noalloc: SM count");
-    d.base = static_cast<char*>(ptr);
-    d.num_sms = sms;
-    d.ready = true;
+    g_noalloc_sms[dev] = sms;
   }
-  *out = &d;
+  *base = static_cast<char*>(ptr);
+  *num_sms = g_noalloc_sms[dev];
   return FLUX_OK;
 }
 
@@ -664,26 +662,27 @@ extern "C" int flux_attn_decode_noalloc(const uint16_t* q, const uint16_t* k_cac
                      scale, 0, nullptr, nullptr};
   int rc = check_decode(a, kNoAllocMaxGroups);
   if (rc != FLUX_OK) return rc;
-  NoAllocDevice* dev = nullptr;
-  if ((rc = noalloc_setup(&dev)) != FLUX_OK) return rc;
+  char* base = nullptr;
+  int num_sms = 0;
+  if ((rc = noalloc_setup(&base, &num_sms)) != FLUX_OK) return rc;
   flux::DecodeLaunch p;
   size_t o_bytes = 0;
-  const size_t need = plan_decode(a, dev->num_sms, &p, &o_bytes);
+  const size_t need = plan_decode(a, num_sms, &p, &o_bytes);
   if (kNoAllocPartOff + need > kNoAllocBytes)
     return fail(FLUX_ERR_SHAPE,
                 "flux_attn_decode_noalloc: %zu bytes of split partials exceed the %zu-byte static "
                 "scratch (use flux_attn_decode with a ctx for this shape)",
                 need, kNoAllocBytes - kNoAllocPartOff);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* err = reinterpret_cast<int*>(dev->base + kNoAllocErrOff);
-  int* tickets = reinterpret_cast<int*>(dev->base + kNoAllocTicketOff);
+  int* err = reinterpret_cast<int*>(base + kNoAllocErrOff);
+  int* tickets = reinterpret_cast<int*>(base + kNoAllocTicketOff);
   // The array keeps the previous call's contents: the error word and this
   // call's tickets must start at zero.
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
   if (e == cudaSuccess)
     e = cudaMemsetAsync(tickets, 0, static_cast<size_t>(B) * Hkv * sizeof(int), s);
   if (e != cudaSuccess) return cuda_fail(e, "flux_attn_decode_noalloc: clear scratch");
-  rc = launch_decode_call(a, p, dev->base + kNoAllocPartOff, o_bytes, tickets,
+  rc = launch_decode_call(a, p, base + kNoAllocPartOff, o_bytes, tickets,
                           flux::DevStatus{err, 2000LL * 1000000LL}, s);
   if (rc != FLUX_OK) return rc;
   if (status && (e = cudaMemcpyAsync(status, err, sizeof(int), cudaMemcpyDeviceToDevice, s)) !=
