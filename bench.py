@@ -3,34 +3,38 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flux|reference]
 
-One step is one pass of the routed prefill hot path over the Qwen3-4B-shaped
-layer workload (B 1, T 32768, Hq 32, Hkv 8, d 128, bf16 N(0,1) with 16 planted
-needles per kv head):
-  flux_route (hidden 32768 x 2560, MLP 5120 -> 512 -> 2, biases put layer 0 on
-  FA and layer 1 on SA) -> flux_build_streaming_mask + flux_build_block_index
-  (block 128, sink 1, window 16) -> flux_attn_prefill for layer 0 (FA) and
-  layer 1 (SA), each reading its routing bit on the device.
-value = TFLOP/s over computed (query, key) pairs of both layers (4 d FLOPs per
-pair per head) / step time.  The decode half of the metric (KV GB/s) is timed
-in the same run on the 36-layer Qwen3-4B-shaped decode workload (batch 16, KV
-131072 + step, 18 FA / 18 SA layers, 64 steps; every layer appends the new token's
-K/V -- the full cache of an FA layer, the compact sink + window ring of an SA layer -- and
-decodes) and reported under "decode", with one SA ring layer timed alone with and
-without an L2 flush.  On one GPU the line also carries, each timed in a few seconds,
-"prefill_36_layers" (the routed 36-layer prefill at T 65536: router, mask, CSR, 36
-layers reading their bits on the device) and "llama_3_1_8b" (32-layer shapes:
-prefill FA and SA layers at T 131072 for windows of 8/16/32 blocks; 32-layer decode
-at B 4, S 131072 for 0-100 % SA layers) and "dynamic_sa" (flux_select_blocks on the
-layer's Q/K, the CSR build and SA prefill over the selected mask, and the planted needles'
-key blocks it keeps); --no-extended skips them.
+One step is one pass of the routed prefill hot path over the 36-layer
+Qwen3-4B-shaped workload (B 1, T 65536, Hq 32, Hkv 8, d 128; every layer has its
+own bf16 N(0,1) Q/K/V resident in HBM, with 16 planted needles per kv head):
+  flux_route (hidden 65536 x 2560, MLP 5120 -> 512 -> 36; the biases put 18 layers
+  on each side with a wide margin) -> flux_build_streaming_mask +
+  flux_build_block_index (block 128, sink 1, window 16) -> 36 flux_attn_prefill
+  launches, each reading its layer's routing bit on the device.
+value = TFLOP/s over the computed (query, key) pairs of all 36 layers (4 d FLOPs
+per pair per query head) / step time.  "roofline" is the FA layer's prefill kernel
+in that step; "roofline_sa_prefill" the SA layer's; "roofline_decode" the decode
+kernel of an FA layer in the decode half of the metric.
 
-Every input is seeded and synthetic; every timed input (640 MB for prefill,
-17 GB of KV for decode) is larger than the 126 MB L2, so no flush is needed.
-Multi-GPU: the units are independent (no exchange), so each rank runs its own
-replica of the step (weak scaling) and rank 0 reports the max time.
+The decode half of the metric (KV GB/s) is timed in the same run on the 36-layer
+Qwen3-4B-shaped decode workload (batch 16, KV 131072 + step, 18 FA / 18 SA layers,
+64 steps; every layer appends the new token's K/V -- the full cache of an FA layer,
+the compact sink + window ring of an SA layer -- and decodes) and reported under
+"decode", with one SA ring layer timed alone with and without an L2 flush.  On one
+GPU the line also carries, each timed in a few seconds: "layer_pair_T32768" (one FA
+and one SA layer of the Qwen3-4B shape at T 32768 with the 2-layer router),
+"soft_prefill", "dynamic_sa" (flux_select_blocks on that layer's Q/K, the CSR build
+and SA prefill over the selected mask) and "llama_3_1_8b" (the 32-layer prefill
+step at T 131072 measured as one step per SA fraction 0/25/50/75/100 % and per
+window 8/16/32 blocks; the 32-layer decode step at B 4, S 131072); --no-extended
+skips them.
 
---impl reference times the oracle (plain fp64 C, OpenMP) on the host cores on
-a bounded sample of the same workload, as the reference arm.
+Every input is seeded and synthetic; every timed input (27 GB of Q/K/V for the
+prefill step, 17 GB of KV for decode) is larger than the 126 MB L2, so no flush is
+needed.  Multi-GPU: the units are independent (no exchange), so each rank runs its
+own replica of the step (weak scaling) and rank 0 reports the max time.
+
+--impl reference times the oracle (plain fp64 C, OpenMP) on the host cores on a
+bounded sample of the same workload, as the reference arm.
 """
 from __future__ import annotations
 
@@ -42,7 +46,6 @@ import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 import numpy as np
@@ -50,10 +53,14 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-T, HQ, HKV, D = 32768, 32, 8, 128
+HQ, HKV, D = 32, 8, 128
 HD, H1 = 2560, 512
 BLOCK, SINK, WIN = 128, 1, 16
+T_STEP, L_STEP = 65536, 36                 # the routed prefill step
+T_PAIR = 32768                              # the single-layer pair (extra)
 DEC_B, DEC_S, DEC_LAYERS, DEC_STEPS = 16, 131072, 36, 64
+# Dense bf16 tensor and HBM figures of the B200 specification, beside the measured peaks.
+SPEC_TFLOPS, SPEC_HBM_GBS = 2250.0, 8000.0
 
 
 def causal_pairs_fa(T):
@@ -197,24 +204,244 @@ def whole_job_rate(units_per_rank: float, world: int, ms: float, scale: float = 
     return units_per_rank * world / (ms * 1e-3) / scale
 
 
+def roofline_entry(achieved, peaks, peak_src, bound, kernel, traffic, algorithmic, per,
+                   long_step=False):
+    """A roofline object: achieved against the measured peak and against the
+    specification's nominal peak.  For the tensor pipe the measured peak is cuBLAS's
+    sustained figure (a seconds-long loop under the power cap) for a kernel timed inside
+    a long step (long_step), else its burst figure; the other one is reported beside it.
+    algorithmic: the kernel's algorithmic FLOPs or bytes per launch."""
+    if bound == "tensor":
+        burst = peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained"))
+        sus = peaks.get("bf16_tflops_sustained", burst)
+        peak = sus if long_step else burst
+        spec, unit = SPEC_TFLOPS, "TFLOP/s"
+        src = f"{peak_src} bf16_tflops{'_sustained' if long_step else ''} " \
+              f"({'sustained: timed inside a seconds-long step' if long_step else 'burst'})"
+    else:
+        peak = peaks["hbm_gbs"]
+        spec, unit = SPEC_HBM_GBS, "GB/s"
+        src = f"{peak_src} hbm_gbs (copy)"
+    out = {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+           "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel,
+           "peak_source": src, "algorithmic_per_launch": algorithmic, "per": per,
+           "frac_of_spec": round(achieved / spec, 4), "spec_peak": spec}
+    if bound == "tensor":
+        if long_step:
+            out["frac_of_burst"] = round(achieved / burst, 4)
+        else:
+            out["frac_of_sustained"] = round(achieved / sus, 4)
+    return out
+
+
 # --------------------------------------------------------------------------- flux arm
 
-class PrefillWorkload:
+def _events(torch, n):
+    return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(n)]
+
+
+class LayerStack:
+    """L attention layers of one model at prompt length T (B 1, Hq 32, Hkv 8, d 128),
+    every layer with its own Q/K/V resident in HBM (bf16 N(0,1) drawn on the device,
+    16 planted needles per kv head when asked), and one output buffer that every layer
+    writes in turn (the next op of a model reads it before the next layer runs)."""
+
+    def __init__(self, ctx, dev, T, L, cfg, salt0=0, needles=True):
+        import torch
+        from sparse_attention_flux_b200 import synth
+        self.ctx, self.dev, self.T, self.L = ctx, dev, T, L
+        self.q, self.k, self.v = [], [], []
+        for l in range(L):
+            q = synth.torch_normal_bf16((1, T, HQ, D), synth.seed_for(cfg, l, salt0 + 1), dev)
+            k = synth.torch_normal_bf16((1, T, HKV, D), synth.seed_for(cfg, l, salt0 + 2), dev)
+            v = synth.torch_normal_bf16((1, T, HKV, D), synth.seed_for(cfg, l, salt0 + 3), dev)
+            if needles:
+                synth.plant_needles_torch(q, k, synth.seed_for(cfg, l, salt0))
+            self.q.append(q)
+            self.k.append(k)
+            self.v.append(v)
+        self.o = torch.empty_like(self.q[0])
+        self.nb = (T + BLOCK - 1) // BLOCK
+        self.scale = 1.0 / math.sqrt(D)
+
+    def flops(self, mode_h, W=WIN):
+        f_fa = 4.0 * D * causal_pairs_fa(self.T) * HQ
+        f_sa = 4.0 * D * pairs_sa(self.T, BLOCK, SINK, W) * HQ
+        return sum(f_fa if m else f_sa for m in mode_h), f_fa, f_sa
+
+    def layers(self, mode, row_ptr, col, evs=None, q=None, k=None, v=None, o=None, stream=None):
+        c = self.ctx
+        for l in range(self.L):
+            if evs is not None:
+                evs[l][0].record()
+            c.attn_prefill(self.q[l] if q is None else q, self.k[l] if k is None else k,
+                           self.v[l] if v is None else v, self.o if o is None else o, self.scale,
+                           layer_mode=mode, layer=l, row_ptr=row_ptr, col=col, block=BLOCK,
+                           stream=stream)
+            if evs is not None:
+                evs[l][1].record()
+
+
+class RoutedPrefill:
+    """The routed prefill step: the 36-layer Qwen3-4B-shaped workload at T 65536.
+    Router on hidden 65536 x 2560 (MLP 5120 -> 512 -> 36; b2 = +4 on 18 layers and -4
+    on the other 18, chosen by a seeded permutation, so 18 layers go to each mode with
+    |z| >= 1.4) -> streaming mask -> CSR -> 36 prefill launches reading their bits."""
+
+    def __init__(self, ctx, dev, rank):
+        import torch
+        from sparse_attention_flux_b200 import synth
+        self.ctx, self.dev = ctx, dev
+        self.stack = LayerStack(ctx, dev, T_STEP, L_STEP, 2, salt0=10 * rank)
+        h, W1, b1, W2, b2 = synth.router_inputs(T_STEP, HD, H1, L_STEP, synth.seed_for(2) + rank,
+                                                coin_bias=4.0, n_positive=L_STEP // 2)
+        self.hidden_h = synth.torch_from_bits(h).pin_memory()
+        self.hidden = self.hidden_h.to(dev)
+        self.W1, self.b1, self.W2, self.b2 = (torch.from_numpy(x).to(dev) for x in (W1, b1, W2, b2))
+        self.mode = torch.zeros(L_STEP, dtype=torch.uint8, device=dev)
+        nb = self.stack.nb
+        self.nb = nb
+        self.mask = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
+        self.row_ptr = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+        self.col = torch.empty(nb * (SINK + WIN), dtype=torch.int32, device=dev)
+        self.launches = 2 + 1 + 3 + L_STEP   # router (pool, MLP), mask, CSR (3), 36 layers
+        self.step()
+        ctx.check()
+        self.mode_h = self.mode.cpu().numpy()
+        self.flops, self.flops_fa, self.flops_sa = self.stack.flops(self.mode_h)
+
+    def head(self, hidden=None, stream=None):
+        c = self.ctx
+        c.route(self.hidden if hidden is None else hidden, self.W1, self.b1, self.W2, self.b2, 0.5,
+                self.mode, stream=stream)
+        c.build_streaming_mask(self.nb, self.nb, SINK, WIN, self.mask, stream=stream)
+        c.build_block_index(self.mask, self.row_ptr, self.col, stream=stream)
+
+    def step(self, evs=None):
+        self.head()
+        self.stack.layers(self.mode, self.row_ptr, self.col, evs)
+
+    # ---- end to end: host buffers in and out
+    def e2e_setup(self):
+        import torch
+        st = self.stack
+        # One layer's inputs in pinned host memory, sent for every layer: every byte
+        # of every layer's Q/K/V crosses PCIe each step (the values do not change the
+        # work).  Two pinned output buffers take the layers' outputs in turn.
+        self.qkv_h = [x.cpu().pin_memory() for x in (st.q[0], st.k[0], st.v[0])]
+        self.o_h = [torch.empty(st.o.shape, dtype=st.o.dtype).pin_memory() for _ in range(2)]
+        self.ins = [[torch.empty_like(x) for x in (st.q[0], st.k[0], st.v[0])] for _ in range(2)]
+        self.outs = [torch.empty_like(st.o) for _ in range(2)]
+        self.hid_d = torch.empty_like(self.hidden)
+
+    @property
+    def h2d_bytes(self):
+        return self.hidden_h.numel() * 2 + L_STEP * sum(x.numel() * 2 for x in self.qkv_h)
+
+    @property
+    def d2h_bytes(self):
+        return L_STEP * self.o_h[0].numel() * 2
+
+    def e2e_pipelined(self, steps):
+        """The step from pinned host memory through the public API, pipelined per layer
+        over three streams: layer n's prefill overlaps layer n+1's host->device copy of
+        Q/K/V and layer n-1's device->host copy of its output (double-buffered device
+        tensors); each step first uploads the router's hidden states.  Returns ms per
+        step, from an event before the first copy to one after the last copy back."""
+        import torch
+        dev, c, st = self.dev, self.ctx, self.stack
+        s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        ev = lambda: torch.cuda.Event(enable_timing=False)
+        h2d, cmp, d2h = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        hid_done, head_done = ev(), ev()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record(s_in)
+        n = 0
+        for k in range(steps):
+            with torch.cuda.stream(s_in):
+                if k:
+                    s_in.wait_event(head_done)
+                self.hid_d.copy_(self.hidden_h, non_blocking=True)
+                hid_done.record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(hid_done)
+                self.head(self.hid_d, stream=s_cmp)
+                head_done.record(s_cmp)
+            for l in range(L_STEP):
+                b = n % 2
+                with torch.cuda.stream(s_in):
+                    if n >= 2:
+                        s_in.wait_event(cmp[b])
+                    for dst, x in zip(self.ins[b], self.qkv_h):
+                        dst.copy_(x, non_blocking=True)
+                    h2d[b].record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(h2d[b])
+                    if n >= 2:
+                        s_cmp.wait_event(d2h[b])
+                    q, kk, v = self.ins[b]
+                    c.attn_prefill(q, kk, v, self.outs[b], st.scale, layer_mode=self.mode,
+                                   layer=l, row_ptr=self.row_ptr, col=self.col, block=BLOCK,
+                                   stream=s_cmp)
+                    cmp[b].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(cmp[b])
+                    self.o_h[b].copy_(self.outs[b], non_blocking=True)
+                    d2h[b].record(s_out)
+                n += 1
+        s_out.wait_stream(s_in)
+        s_out.wait_stream(s_cmp)
+        t1.record(s_out)
+        t1.synchronize()
+        return t0.elapsed_time(t1) / steps
+
+    def copy_floor_ms(self, reps=2):
+        """ms for one step's host<->device traffic alone: every upload on one stream and
+        every download on another, concurrently (no compute) -- the floor of the
+        pipelined e2e step on this machine's PCIe link."""
+        import torch
+        s_in, s_out = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s_in)
+        s_out.wait_stream(s_in)
+        for _ in range(reps):
+            with torch.cuda.stream(s_in):
+                self.hid_d.copy_(self.hidden_h, non_blocking=True)
+                for l in range(L_STEP):
+                    for dst, x in zip(self.ins[l % 2], self.qkv_h):
+                        dst.copy_(x, non_blocking=True)
+            with torch.cuda.stream(s_out):
+                for l in range(L_STEP):
+                    self.o_h[l % 2].copy_(self.outs[l % 2], non_blocking=True)
+        s_in.wait_stream(s_out)
+        b.record(s_in)
+        b.synchronize()
+        return a.elapsed_time(b) / reps
+
+    def release(self):
+        for name in ("stack", "ins", "outs", "hid_d", "qkv_h", "o_h", "hidden", "hidden_h"):
+            if hasattr(self, name):
+                delattr(self, name)
+
+
+class LayerPair:
+    """One FA and one SA layer of the Qwen3-4B shape at T 32768 (B 1, needles), routed
+    by a 2-logit router on hidden 32768 x 2560 (layer 0 FA, layer 1 SA)."""
+
     def __init__(self, ctx, seed, dev):
         import torch
         from sparse_attention_flux_b200 import synth
         self.ctx, self.dev = ctx, dev
-        g = torch.Generator(device=dev)
+        T = T_PAIR
         q, k, v = synth.attention_inputs(1, T, HQ, HKV, D, seed)
         self.needles = synth.plant_needles_np(q, k, seed)
-        self.q_h = synth.torch_from_bits(q).pin_memory()
-        self.k_h = synth.torch_from_bits(k).pin_memory()
-        self.v_h = synth.torch_from_bits(v).pin_memory()
-        self.q, self.k, self.v = (x.to(dev) for x in (self.q_h, self.k_h, self.v_h))
+        self.q, self.k, self.v = (synth.torch_from_bits(x).to(dev) for x in (q, k, v))
         hidden, W1, b1, W2, b2 = synth.router_inputs(T, HD, H1, 2, seed + 50)
         b2[:] = np.array([4.0, -4.0], np.float32)   # layer 0 -> FA, layer 1 -> SA
-        self.hidden_h = synth.torch_from_bits(hidden).pin_memory()
-        self.hidden = self.hidden_h.to(dev)
+        self.hidden = synth.torch_from_bits(hidden).to(dev)
         self.W1, self.b1, self.W2, self.b2 = (torch.from_numpy(x).to(dev) for x in (W1, b1, W2, b2))
         self.mode = torch.zeros(2, dtype=torch.uint8, device=dev)
         self.nb = T // BLOCK
@@ -222,11 +449,9 @@ class PrefillWorkload:
         self.row_ptr = torch.empty(self.nb + 1, dtype=torch.int32, device=dev)
         self.col = torch.empty(self.nb * (SINK + WIN), dtype=torch.int32, device=dev)
         self.o = [torch.empty_like(self.q) for _ in range(2)]
-        self.o_h = [torch.empty_like(self.q_h).pin_memory() for _ in range(2)]
         self.flops_fa = 4.0 * D * causal_pairs_fa(T) * HQ
         self.flops_sa = 4.0 * D * pairs_sa(T, BLOCK, SINK, WIN) * HQ
         self.flops = self.flops_fa + self.flops_sa
-        self.launches = 2 + 1 + 3 + 2
         self.scale = 1.0 / math.sqrt(D)
 
     def step(self, events=None):
@@ -242,105 +467,31 @@ class PrefillWorkload:
             if events:
                 events[layer][1].record()
 
-    def step_e2e(self):
-        # Host buffers in, host buffers out: the copies are inside the timed region.
-        for dst, src in ((self.q, self.q_h), (self.k, self.k_h), (self.v, self.v_h),
-                         (self.hidden, self.hidden_h)):
-            dst.copy_(src, non_blocking=True)
-        self.step()
-        for l in (0, 1):
-            self.o_h[l].copy_(self.o[l], non_blocking=True)
-
-    def copy_floor_ms(self, reps=5):
-        """ms for one step's host<->device traffic alone: the inputs' upload and the two
-        outputs' download running concurrently on two streams (no compute) -- the floor
-        of the pipelined e2e step on this machine's PCIe link."""
+    def measure(self, steps=5):
         import torch
-        s_in, s_out = torch.cuda.Stream(self.dev), torch.cuda.Stream(self.dev)
-        src = (self.q_h, self.k_h, self.v_h, self.hidden_h)
-        dst = (self.q, self.k, self.v, self.hidden)
-
-        def once():
-            with torch.cuda.stream(s_in):
-                for d_, x in zip(dst, src):
-                    d_.copy_(x, non_blocking=True)
-            with torch.cuda.stream(s_out):
-                for l in (0, 1):
-                    self.o_h[l].copy_(self.o[l], non_blocking=True)
-        once()
-        torch.cuda.synchronize()
+        for _ in range(2):
+            self.step()
+        evs = [_events(torch, 2) for _ in range(steps)]
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        for _ in range(reps):
-            torch.cuda.current_stream().wait_stream(s_in)
-            torch.cuda.current_stream().wait_stream(s_out)
-            s_in.wait_stream(torch.cuda.current_stream())
-            s_out.wait_stream(torch.cuda.current_stream())
-            once()
-        torch.cuda.current_stream().wait_stream(s_in)
-        torch.cuda.current_stream().wait_stream(s_out)
+        for e in evs:
+            self.step(e)
         b.record()
         b.synchronize()
-        return a.elapsed_time(b) / reps
-
-    def e2e_pipelined(self, steps):
-        """The step from pinned host memory, pipelined over three streams: step k's compute
-        overlaps step k+1's host->device copy of its inputs and step k-1's device->host copy
-        of its two outputs (double-buffered device tensors).  Returns ms per step, from an
-        event before the first copy to one after the last copy back."""
-        import torch
-        dev = self.dev
-        s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-        ins = [[torch.empty_like(x) for x in (self.q, self.k, self.v, self.hidden)] for _ in range(2)]
-        outs = [[torch.empty_like(self.q) for _ in range(2)] for _ in range(2)]
-        new_ev = lambda: torch.cuda.Event(enable_timing=False)
-        h2d_done = [new_ev() for _ in range(2)]
-        cmp_done = [new_ev() for _ in range(2)]
-        d2h_done = [new_ev() for _ in range(2)]
-        src = (self.q_h, self.k_h, self.v_h, self.hidden_h)
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        t0.record(s_in)
-        for k in range(steps):
-            b = k % 2
-            with torch.cuda.stream(s_in):
-                if k >= 2:
-                    s_in.wait_event(cmp_done[b])
-                for dst, x in zip(ins[b], src):
-                    dst.copy_(x, non_blocking=True)
-                h2d_done[b].record(s_in)
-            with torch.cuda.stream(s_cmp):
-                s_cmp.wait_event(h2d_done[b])
-                if k >= 2:
-                    s_cmp.wait_event(d2h_done[b])
-                q, kk, v, hid = ins[b]
-                c = self.ctx
-                c.route(hid, self.W1, self.b1, self.W2, self.b2, 0.5, self.mode, stream=s_cmp)
-                c.build_streaming_mask(self.nb, self.nb, SINK, WIN, self.mask, stream=s_cmp)
-                c.build_block_index(self.mask, self.row_ptr, self.col, stream=s_cmp)
-                for layer in (0, 1):
-                    c.attn_prefill(q, kk, v, outs[b][layer], self.scale, layer_mode=self.mode,
-                                   layer=layer, row_ptr=self.row_ptr, col=self.col, block=BLOCK,
-                                   stream=s_cmp)
-                cmp_done[b].record(s_cmp)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(cmp_done[b])
-                for layer in (0, 1):
-                    self.o_h[layer].copy_(outs[b][layer], non_blocking=True)
-                d2h_done[b].record(s_out)
-        s_out.wait_stream(s_in)
-        s_out.wait_stream(s_cmp)
-        t1.record(s_out)
-        t1.synchronize()
-        return t0.elapsed_time(t1) / steps
-
-    @property
-    def h2d_bytes(self):
-        return sum(x.numel() * 2 for x in (self.q_h, self.k_h, self.v_h, self.hidden_h))
-
-    @property
-    def d2h_bytes(self):
-        return sum(x.numel() * 2 for x in self.o_h)
+        self.ctx.check()
+        ms = a.elapsed_time(b) / steps
+        fa = statistics.mean(e[0][0].elapsed_time(e[0][1]) for e in evs)
+        sa = statistics.mean(e[1][0].elapsed_time(e[1][1]) for e in evs)
+        return {"workload": "qwen3-4b-layer-pair: B 1, T 32768, Hq 32, Hkv 8, d 128, needles; "
+                            "router 32768x2560 -> MLP 5120-512-2 (layer 0 FA, layer 1 SA); "
+                            "SA block 128, sink 1, window 16",
+                "ms_per_step": round(ms, 4),
+                "TFLOP/s": round(self.flops / (ms * 1e-3) / 1e12, 1),
+                "fa_layer": {"ms": round(fa, 4),
+                             "TFLOP/s": round(self.flops_fa / (fa * 1e-3) / 1e12, 1)},
+                "sa_layer": {"ms": round(sa, 4),
+                             "TFLOP/s": round(self.flops_sa / (sa * 1e-3) / 1e12, 1)},
+                "timed_steps": steps}
 
 
 class DecodeWorkload:
@@ -502,182 +653,6 @@ class DecodeWorkload:
                                              BLOCK)
 
 
-def _events(torch, n):
-    return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(n)]
-
-
-def prefill_36_layers(ctx, dev, seed, reps=2):
-    """36-layer routed prefill, Qwen3-4B shapes at T 65536 (B 1, Hq 32, Hkv 8, d 128):
-    router on hidden 65536 x 2560 (MLP 5120 -> 512 -> 36, b2 = +-2 from a seeded coin:
-    about half the layers SA) -> mask -> CSR -> 36 flux_attn_prefill calls, each reading
-    its layer's bit on the device.  Q/K/V are aliased across layers (805 MB, far above
-    L2); the values do not change the work.  One warm-up pass, then `reps` timed passes."""
-    import torch
-    from sparse_attention_flux_b200 import synth
-    T2, L = 65536, 36
-    q = synth.torch_normal_bf16((1, T2, HQ, D), seed + 1, dev)
-    k = synth.torch_normal_bf16((1, T2, HKV, D), seed + 2, dev)
-    v = synth.torch_normal_bf16((1, T2, HKV, D), seed + 3, dev)
-    o = torch.empty_like(q)
-    h, W1, b1, W2, b2 = synth.router_inputs(T2, HD, H1, L, seed + 4, coin_bias=2.0)
-    hidden = synth.torch_from_bits(h).to(dev)
-    W1, b1, W2, b2 = (torch.from_numpy(x).to(dev) for x in (W1, b1, W2, b2))
-    del h
-    mode = torch.empty(L, dtype=torch.uint8, device=dev)
-    nb = T2 // BLOCK
-    mask = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
-    row_ptr = torch.empty(nb + 1, dtype=torch.int32, device=dev)
-    col = torch.empty(nb * nb, dtype=torch.int32, device=dev)
-    scale = 1.0 / math.sqrt(D)
-
-    def one(evs=None):
-        if evs is not None:
-            evs[0][0].record()
-        ctx.route(hidden, W1, b1, W2, b2, 0.5, mode)
-        ctx.build_streaming_mask(nb, nb, SINK, WIN, mask)
-        ctx.build_block_index(mask, row_ptr, col)
-        if evs is not None:
-            evs[0][1].record()
-        for layer in range(L):
-            if evs is not None:
-                evs[1 + layer][0].record()
-            ctx.attn_prefill(q, k, v, o, scale, layer_mode=mode, layer=layer, row_ptr=row_ptr,
-                             col=col, block=BLOCK)
-            if evs is not None:
-                evs[1 + layer][1].record()
-
-    one()
-    ctx.check()
-    runs = [_events(torch, 1 + L) for _ in range(reps)]
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for evs in runs:
-        one(evs)
-    b.record()
-    b.synchronize()
-    ctx.check()
-    step_ms = a.elapsed_time(b) / reps
-    mode_h = mode.cpu().numpy()
-    fa_l = [l for l in range(L) if mode_h[l]]
-    sa_l = [l for l in range(L) if not mode_h[l]]
-    per = [[evs[1 + l][0].elapsed_time(evs[1 + l][1]) for l in range(L)] for evs in runs]
-    fa_ms = statistics.mean(p[l] for p in per for l in fa_l) if fa_l else 0.0
-    sa_ms = statistics.mean(p[l] for p in per for l in sa_l) if sa_l else 0.0
-    head_ms = statistics.mean(evs[0][0].elapsed_time(evs[0][1]) for evs in runs)
-    f_fa = 4.0 * D * causal_pairs_fa(T2) * HQ
-    f_sa = 4.0 * D * pairs_sa(T2, BLOCK, SINK, WIN) * HQ
-    flops = len(fa_l) * f_fa + len(sa_l) * f_sa
-    out = {
-        "workload": "qwen3-4b-36L-routed-prefill: B 1, T 65536, Hq 32, Hkv 8, d 128; router "
-                    "65536x2560 -> MLP 5120-512-36 (b2 = +-2, seeded coin); SA block 128, "
-                    "sink 1, window 16; Q/K/V aliased across layers",
-        "fa_layers": len(fa_l), "sa_layers": len(sa_l),
-        "ms_per_step": round(step_ms, 3),
-        "TFLOP/s": round(flops / (step_ms * 1e-3) / 1e12, 1),
-        "fa_layer": {"ms": round(fa_ms, 3),
-                     "TFLOP/s": round(f_fa / (fa_ms * 1e-3) / 1e12, 1) if fa_ms else None},
-        "sa_layer": {"ms": round(sa_ms, 3),
-                     "TFLOP/s": round(f_sa / (sa_ms * 1e-3) / 1e12, 1) if sa_ms else None},
-        "router_mask_csr_us": round(head_ms * 1e3, 1),
-        "timed_passes": reps,
-    }
-    del q, k, v, o, hidden
-    torch.cuda.empty_cache()
-    return out
-
-
-def llama_sweep(ctx, dev, seed):
-    """Llama-3.1-8B shapes (32 layers, Hq 32, Hkv 8, d 128), no router (fixed modes).
-
-    prefill, B 1, T 131072: one FA layer and one SA layer per window W in {8, 16, 32}
-    blocks of 128 (sink 1), each timed over 2 launches after a warm-up; the 32-layer step
-    at each SA fraction is the sum of its layers' measured times (layers are sequential,
-    independent launches whose inputs exceed L2).
-    decode, B 4, S 131072: the whole 32-layer step measured at SA fractions 0/25/50/75/100 %
-    (W 16; seeded layer choice) and at 50 % for W 8 and 32; every layer has its own full
-    cache (2.15 GB; 69 GB in all), so no layer's window is left in L2 by another's."""
-    import torch
-    from sparse_attention_flux_b200 import synth
-    L, T3, B4, S4 = 32, 131072, 4, 131072
-    scale = 1.0 / math.sqrt(D)
-    out = {"workload": "llama-3.1-8b: 32 layers, Hq 32, Hkv 8, d 128; prefill B 1 T 131072; "
-                       "decode B 4 S 131072; sink 1, W in {8, 16, 32} blocks of 128"}
-    # ---- prefill
-    q = synth.torch_normal_bf16((1, T3, HQ, D), seed + 1, dev)
-    k = synth.torch_normal_bf16((1, T3, HKV, D), seed + 2, dev)
-    v = synth.torch_normal_bf16((1, T3, HKV, D), seed + 3, dev)
-    o = torch.empty_like(q)
-    nb = T3 // BLOCK
-    mask = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
-    row_ptr = torch.empty(nb + 1, dtype=torch.int32, device=dev)
-    col = torch.empty(nb * nb, dtype=torch.int32, device=dev)
-    fa_mode = torch.ones(1, dtype=torch.uint8, device=dev)
-    sa_mode = torch.zeros(1, dtype=torch.uint8, device=dev)
-
-    def timed(fn, n=2):
-        fn()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(n):
-            fn()
-        b.record()
-        b.synchronize()
-        return a.elapsed_time(b) / n
-
-    ctx.build_streaming_mask(nb, nb, SINK, 16, mask)
-    ctx.build_block_index(mask, row_ptr, col)
-    fa_ms = timed(lambda: ctx.attn_prefill(q, k, v, o, scale, layer_mode=fa_mode, row_ptr=row_ptr,
-                                           col=col, block=BLOCK))
-    f_fa = 4.0 * D * causal_pairs_fa(T3) * HQ
-    pre = {"fa_layer": {"ms": round(fa_ms, 3), "TFLOP/s": round(f_fa / (fa_ms * 1e-3) / 1e12, 1)}}
-    sa_ms_w = {}
-    for W in (8, 16, 32):
-        ctx.build_streaming_mask(nb, nb, SINK, W, mask)
-        ctx.build_block_index(mask, row_ptr, col)
-        sa_ms_w[W] = timed(lambda: ctx.attn_prefill(q, k, v, o, scale, layer_mode=sa_mode,
-                                                    row_ptr=row_ptr, col=col, block=BLOCK))
-        f_sa = 4.0 * D * pairs_sa(T3, BLOCK, SINK, W) * HQ
-        pre[f"sa_layer_W{W}"] = {"ms": round(sa_ms_w[W], 3),
-                                 "TFLOP/s": round(f_sa / (sa_ms_w[W] * 1e-3) / 1e12, 1)}
-    ctx.check()
-    pre["step_ms_by_sa_fraction_W16"] = {
-        f"{pct}%": round((L - L * pct // 100) * fa_ms + (L * pct // 100) * sa_ms_w[16], 1)
-        for pct in (0, 25, 50, 75, 100)}
-    pre["how"] = "per-layer launches timed; 32-layer step = sum of its layers' times"
-    out["prefill"] = pre
-    del q, k, v, o
-    torch.cuda.empty_cache()
-    # ---- decode
-    shape = (B4, S4, HKV, D)
-    caches = [(synth.torch_normal_bf16(shape, seed + 10 * i + 11, dev),
-               synth.torch_normal_bf16(shape, seed + 10 * i + 12, dev)) for i in range(L)]
-    qd = synth.torch_normal_bf16((B4, HQ, D), seed + 30, dev)
-    od = torch.empty_like(qd)
-    sl = torch.full((B4,), S4, dtype=torch.int32, device=dev)
-    kv_row = HKV * D * 2 * 2
-
-    def dec_step(mode_t, W):
-        for layer in range(L):
-            kc, vc = caches[layer]
-            ctx.attn_decode(qd, kc, vc, sl, od, scale, layer_mode=mode_t, layer=layer,
-                            sink_blocks=SINK, window_blocks=W, block=BLOCK)
-
-    dec = {}
-    for pct, W in [(0, 16), (25, 16), (50, 16), (75, 16), (100, 16), (50, 8), (50, 32)]:
-        n_sa = L * pct // 100
-        mode_t = torch.from_numpy(synth.layer_mode_choice(L, L - n_sa, seed + pct)).to(dev)
-        ms = timed(lambda: dec_step(mode_t, W), n=5)
-        byts = B4 * ((L - n_sa) * S4 + n_sa * sa_decode_tokens(S4, BLOCK, SINK, W)) * kv_row
-        dec[f"sa{pct}%_W{W}"] = {"ms_per_step": round(ms, 3),
-                                 "GB/s": round(byts / (ms * 1e-3) / 1e9, 1)}
-    ctx.check()
-    out["decode"] = dec
-    del caches
-    torch.cuda.empty_cache()
-    return out
-
-
 def dynamic_sa(ctx, wl, dev, reps=5):
     """Dynamic SA block selection on the bench layer's own Q and K (flux_select_blocks:
     strided antidiagonal block scores, stride 8, then the fewest blocks after the sink
@@ -715,7 +690,7 @@ def dynamic_sa(ctx, wl, dev, reps=5):
     kept = int(m.sum())
     pairs = (kept - int(np.trace(m))) * BLOCK * BLOCK + nb * BLOCK * (BLOCK + 1) // 2
     flops_sa = 4.0 * D * pairs * HQ
-    nr = T // S
+    nr = T_PAIR // S
     flops_sel = 2.0 * S * D * (nr * (nr + 1) / 2) * HQ
     hit_dyn = hit_st = total = 0
     for (_h, r, pos) in wl.needles:
@@ -741,17 +716,120 @@ def dynamic_sa(ctx, wl, dev, reps=5):
     }
 
 
+def llama_sweep(ctx, dev, rank, hbm_gbs):
+    """Llama-3.1-8B shapes (32 layers, Hq 32, Hkv 8, d 128), no router (fixed modes from
+    a seeded layer choice).
+
+    prefill, B 1, T 131072, every layer with its own Q/K/V (48 GB resident): the whole
+    32-layer step (mask + CSR + 32 launches reading their bits on the device) measured
+    once per SA fraction 0/25/50/75/100 % at W 16 and at 50 % for W 8 and 32, after one
+    warm-up step; per-layer CUDA events give the FA and SA layer rates inside it.
+    decode, B 4, S 131072: the whole 32-layer step measured at SA fractions
+    0/25/50/75/100 % (W 16) and at 50 % for W 8 and 32; every layer has its own full
+    cache (2.15 GB; 69 GB in all), so no layer's window is left in L2 by another's."""
+    import torch
+    from sparse_attention_flux_b200 import synth
+    L, T3, B4, S4 = 32, 131072, 4, 131072
+    scale = 1.0 / math.sqrt(D)
+    out = {"workload": "llama-3.1-8b: 32 layers, Hq 32, Hkv 8, d 128; prefill B 1 T 131072 "
+                       "(per-layer Q/K/V resident); decode B 4 S 131072; sink 1, W in {8, 16, 32} "
+                       "blocks of 128"}
+    # ---- prefill
+    st = LayerStack(ctx, dev, T3, L, 4, salt0=10 * rank, needles=False)
+    nb = st.nb
+    mask = torch.empty((nb, nb), dtype=torch.uint8, device=dev)
+    row_ptr = torch.empty(nb + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(nb * (SINK + 32), dtype=torch.int32, device=dev)
+
+    def step(mode_t, W, evs=None):
+        ctx.build_streaming_mask(nb, nb, SINK, W, mask)
+        ctx.build_block_index(mask, row_ptr, col)
+        st.layers(mode_t, row_ptr, col, evs)
+
+    pre = {}
+    warmed = False
+    for pct, W in [(0, 16), (25, 16), (50, 16), (75, 16), (100, 16), (50, 8), (50, 32)]:
+        n_sa = L * pct // 100
+        mode_h = synth.layer_mode_choice(L, L - n_sa, synth.seed_for(4) + pct)
+        mode_t = torch.from_numpy(mode_h).to(dev)
+        if not warmed:
+            step(mode_t, W)
+            warmed = True
+        evs = _events(torch, L)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step(mode_t, W, evs)
+        b.record()
+        b.synchronize()
+        ctx.check()
+        ms = a.elapsed_time(b)
+        flops, f_fa, f_sa = st.flops(mode_h, W)
+        per = [x.elapsed_time(y) for x, y in evs]
+        fa_ms = [per[l] for l in range(L) if mode_h[l]]
+        sa_ms = [per[l] for l in range(L) if not mode_h[l]]
+        ent = {"ms_per_step": round(ms, 2), "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1)}
+        if fa_ms:
+            ent["fa_layer_TFLOP/s"] = round(f_fa / (statistics.mean(fa_ms) * 1e-3) / 1e12, 1)
+        if sa_ms:
+            ent["sa_layer_ms"] = round(statistics.mean(sa_ms), 3)
+            ent["sa_layer_TFLOP/s"] = round(f_sa / (statistics.mean(sa_ms) * 1e-3) / 1e12, 1)
+        pre[f"sa{pct}%_W{W}"] = ent
+    pre["how"] = ("one measured 32-layer step per entry (mask + CSR + 32 prefill launches), "
+                  "CUDA events around the step and around each layer's launch")
+    out["prefill"] = pre
+    del st
+    torch.cuda.empty_cache()
+    # ---- decode
+    shape = (B4, S4, HKV, D)
+    caches = [(synth.torch_normal_bf16(shape, synth.seed_for(4, l, 4) + rank, dev),
+               synth.torch_normal_bf16(shape, synth.seed_for(4, l, 5) + rank, dev)) for l in range(L)]
+    qd = synth.torch_normal_bf16((B4, HQ, D), synth.seed_for(4, 0, 6) + rank, dev)
+    od = torch.empty_like(qd)
+    sl = torch.full((B4,), S4, dtype=torch.int32, device=dev)
+    kv_row = HKV * D * 2 * 2
+
+    def dec_step(mode_t, W):
+        for layer in range(L):
+            kc, vc = caches[layer]
+            ctx.attn_decode(qd, kc, vc, sl, od, scale, layer_mode=mode_t, layer=layer,
+                            sink_blocks=SINK, window_blocks=W, block=BLOCK)
+
+    def timed(fn, n):
+        fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / n
+
+    dec = {}
+    for pct, W in [(0, 16), (25, 16), (50, 16), (75, 16), (100, 16), (50, 8), (50, 32)]:
+        n_sa = L * pct // 100
+        mode_t = torch.from_numpy(synth.layer_mode_choice(L, L - n_sa, synth.seed_for(4) + pct)).to(dev)
+        ms = timed(lambda: dec_step(mode_t, W), 5)
+        byts = B4 * ((L - n_sa) * S4 + n_sa * sa_decode_tokens(S4, BLOCK, SINK, W)) * kv_row
+        dec[f"sa{pct}%_W{W}"] = {"ms_per_step": round(ms, 3),
+                                 "GB/s": round(byts / (ms * 1e-3) / 1e9, 1),
+                                 "frac_of_hbm": round(byts / (ms * 1e-3) / 1e9 / hbm_gbs, 4)}
+    ctx.check()
+    out["decode"] = dec
+    del caches
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_flux(args, rank, world, dev_index):
     import torch
-    import torch.distributed as dist
+    from sparse_attention_flux_b200 import synth
     from sparse_attention_flux_b200.flux import Context
 
     torch.cuda.set_device(dev_index)
     dev = torch.device("cuda", dev_index)
     peaks, peak_src = load_peaks()
     ctx = Context(dev_index, 512 << 20)
-    from sparse_attention_flux_b200 import synth
-    wl = PrefillWorkload(ctx, synth.seed_for(1) + 1000 * rank, dev)
+    wl = RoutedPrefill(ctx, dev, rank)
 
     barrier = lambda: dist_barrier(world)
     ranks_max = lambda x: max_over_ranks(x, world, dev)
@@ -759,10 +837,10 @@ def run_flux(args, rank, world, dev_index):
     for _ in range(args.warmup):
         wl.step()
     ctx.check()
-    # Per-kernel CUDA events on the launching (current) stream, read after the
-    # loop so that no host synchronisation sits inside the timed region.
+    # Per-layer CUDA events on the launching (current) stream, read after the loop so
+    # that no host synchronisation sits inside the timed region.
     new_ev = lambda: torch.cuda.Event(enable_timing=True)
-    evs = [[[new_ev(), new_ev()] for _ in range(2)] for _ in range(args.steps)]
+    evs = [_events(torch, L_STEP) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev_index) as clk:
@@ -773,93 +851,93 @@ def run_flux(args, rank, world, dev_index):
         stop.record()
         torch.cuda.synchronize()
     barrier()
-    fa_ms = [e[0][0].elapsed_time(e[0][1]) for e in evs]
-    sa_ms = [e[1][0].elapsed_time(e[1][1]) for e in evs]
     total_ms = start.elapsed_time(stop)
     ctx.check()
     clocks = clk.summary()
+    if not np.array_equal(wl.mode.cpu().numpy(), wl.mode_h):
+        raise RuntimeError("routing changed between steps")
+    fa_l = [l for l in range(L_STEP) if wl.mode_h[l]]
+    sa_l = [l for l in range(L_STEP) if not wl.mode_h[l]]
+    per = [[a.elapsed_time(b) for a, b in e] for e in evs]
+    fa_avg = statistics.mean(p[l] for p in per for l in fa_l)
+    sa_avg = statistics.mean(p[l] for p in per for l in sa_l)
+    layers_ms = statistics.mean(sum(p) for p in per)
     total_ms = ranks_max(total_ms)
     ms_per_step = total_ms / args.steps
     value = whole_job_rate(wl.flops, world, ms_per_step)
+    fa_tflops = wl.flops_fa / (fa_avg * 1e-3) / 1e12
+    sa_tflops = wl.flops_sa / (sa_avg * 1e-3) / 1e12
+    fa_bytes = 2 * (2 * T_STEP * HQ * D + 2 * T_STEP * HKV * D)    # Q, O + K, V (bf16)
 
-    # e2e: host buffers in and out through the same public API, copies inside the timed
-    # region -- pipelined over three streams, and serial for reference.
-    e2e_steps = max(4, args.steps)   # the same K steps as the device-timed region
-    wl.e2e_pipelined(2)
-    barrier()
-    e2e_ms = ranks_max(wl.e2e_pipelined(e2e_steps))
-    e2e_value = whole_job_rate(wl.flops, world, e2e_ms)
-    for _ in range(max(1, args.warmup // 2)):
-        wl.step_e2e()
-    torch.cuda.synchronize()
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record()
-    for _ in range(e2e_steps):
-        wl.step_e2e()
-    s1.record()
-    s1.synchronize()
-    e2e_serial_ms = ranks_max(s0.elapsed_time(s1) / e2e_steps)
-    e2e_serial_value = whole_job_rate(wl.flops, world, e2e_serial_ms)
-    copy_floor = wl.copy_floor_ms()
-
-    # router latency: the step's router, and the 36-layer router (hidden 65536 x 2560,
-    # MLP 5120 -> 512 -> 36); CUDA events around 20 back-to-back calls.
-    def time_router(hid, W1, b1, W2, b2, mode):
-        ctx.route(hid, W1, b1, W2, b2, 0.5, mode)
+    # router latency on the step's router (hidden 65536 x 2560, MLP 5120 -> 512 -> 36)
+    def time_router():
+        ctx.route(wl.hidden, wl.W1, wl.b1, wl.W2, wl.b2, 0.5, wl.mode)
         a_, b_ = new_ev(), new_ev()
         a_.record()
         for _ in range(20):
-            ctx.route(hid, W1, b1, W2, b2, 0.5, mode)
+            ctx.route(wl.hidden, wl.W1, wl.b1, wl.W2, wl.b2, 0.5, wl.mode)
         b_.record()
         b_.synchronize()
         return a_.elapsed_time(b_) / 20 * 1e3
-    router_us = time_router(wl.hidden, wl.W1, wl.b1, wl.W2, wl.b2, wl.mode)
-    h36, W1_36, b1_36, W2_36, b2_36 = synth.router_inputs(65536, HD, H1, 36, synth.seed_for(2),
-                                                          coin_bias=2.0)
-    mode36 = torch.empty(36, dtype=torch.uint8, device=dev)
-    router36_us = time_router(synth.torch_from_bits(h36).to(dev),
-                              *(torch.from_numpy(x).to(dev) for x in (W1_36, b1_36, W2_36, b2_36)),
-                              mode36)
-    del h36
+    router_us = time_router()
 
-    # soft-routing forward blend on the same layer: FA pass + SA pass with a blend epilogue
-    score = torch.tensor([0.3], dtype=torch.float32, device=dev)
-    soft = lambda: ctx.attn_prefill_soft(wl.q, wl.k, wl.v, wl.o[0], wl.scale, score, 0,
-                                         wl.row_ptr, wl.col, BLOCK)
-    soft()
-    s0, s1 = new_ev(), new_ev()
-    s0.record()
-    for _ in range(3):
-        soft()
-    s1.record()
-    s1.synchronize()
-    soft_ms = s0.elapsed_time(s1) / 3
-    soft_line = {"ms": round(soft_ms, 4), "TFLOP/s": round(wl.flops / (soft_ms * 1e-3) / 1e12, 1),
-                 "note": "flux_attn_prefill_soft, r = 0.3: FA + SA passes, blended in the SA epilogue"}
-
-    dyn_line = dynamic_sa(ctx, wl, dev) if (world == 1 and not args.no_extended) else None
-
-    h2d_bytes, d2h_bytes, launches = wl.h2d_bytes, wl.d2h_bytes, wl.launches * args.steps
-    fa_avg = statistics.mean(fa_ms)
-    sa_avg = statistics.mean(sa_ms)
-    # The timed region is short (about 20 steps of 9 ms) and runs at the maximum SM clock
-    # (sampled below), so the kernel is compared with cuBLAS's burst figure; the sustained
-    # figure (a seconds-long loop settled under the power cap, at about 1.3 GHz) is context.
-    peak_t = peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained"))
-    peak_sus = peaks.get("bf16_tflops_sustained", peak_t)
-    fa_tflops = wl.flops_fa / (fa_avg * 1e-3) / 1e12
-    sa_tflops = wl.flops_sa / (sa_avg * 1e-3) / 1e12
-
-    # decode half of the metric
+    # e2e: host buffers in and out through the same public API, copies inside the timed
+    # region, pipelined per layer over three streams.
+    wl.e2e_setup()
+    e2e_steps = args.steps
+    wl.e2e_pipelined(1)
+    barrier()
+    e2e_ms = ranks_max(wl.e2e_pipelined(e2e_steps))
+    ctx.check()
+    e2e_value = whole_job_rate(wl.flops, world, e2e_ms)
+    copy_floor = wl.copy_floor_ms()
+    h2d_bytes, d2h_bytes = wl.h2d_bytes, wl.d2h_bytes
+    launches = wl.launches * args.steps
+    step_line = {"fa_layers": len(fa_l), "sa_layers": len(sa_l),
+                 "fa_layer": {"ms": round(fa_avg, 3), "TFLOP/s": round(fa_tflops, 1)},
+                 "sa_layer": {"ms": round(sa_avg, 4), "TFLOP/s": round(sa_tflops, 1)},
+                 "router_mask_csr_ms": round(ms_per_step - layers_ms, 4),
+                 "router_us": round(router_us, 2),
+                 "router_context": "pages: 0.20 ms per layer for their router (hardware not stated)",
+                 "resident_qkv_gb": round(sum(x.numel() * 2 for x in wl.stack.q + wl.stack.k +
+                                              wl.stack.v) / 1e9, 2),
+                 "flops_per_step": wl.flops}
+    wl.release()
     del wl
     torch.cuda.empty_cache()
-    dec = None
+
+    extra = {}
+    # ---- the single-layer pair at T 32768, the soft blend and dynamic SA on it
+    if not args.no_extended and world == 1:
+        pair = LayerPair(ctx, synth.seed_for(1), dev)
+        extra["layer_pair_T32768"] = pair.measure()
+        score = torch.tensor([0.3], dtype=torch.float32, device=dev)
+        soft = lambda: ctx.attn_prefill_soft(pair.q, pair.k, pair.v, pair.o[0], pair.scale, score,
+                                             0, pair.row_ptr, pair.col, BLOCK)
+        soft()
+        s0, s1 = new_ev(), new_ev()
+        s0.record()
+        for _ in range(3):
+            soft()
+        s1.record()
+        s1.synchronize()
+        soft_ms = s0.elapsed_time(s1) / 3
+        extra["soft_prefill"] = {
+            "ms": round(soft_ms, 4), "TFLOP/s": round(pair.flops / (soft_ms * 1e-3) / 1e12, 1),
+            "note": "flux_attn_prefill_soft on the T 32768 layer, r = 0.3: FA + SA passes, "
+                    "blended in the SA epilogue"}
+        extra["dynamic_sa"] = dynamic_sa(ctx, pair, dev)
+        del pair
+        torch.cuda.empty_cache()
+
+    # ---- decode half of the metric
+    dec = roof_dec = None
     if not args.no_decode:
         dw = DecodeWorkload(ctx, synth.seed_for(3) + 1000 * rank, dev, args.decode_steps)
         for s in range(min(3, dw.steps)):
             dw.step(s)
         ctx.check()
-        # eager steps: per-kernel events for the FA layer (and the eager step time)
+        # eager steps: per-kernel events for the first FA layer (and the eager step time)
         fevs = [(new_ev(), new_ev()) for _ in range(dw.steps)]
         torch.cuda.synchronize()
         e0, e1 = new_ev(), new_ev()
@@ -870,7 +948,6 @@ def run_flux(args, rank, world, dev_index):
         e1.synchronize()
         fa_dec_ms = [a_.elapsed_time(b_) for a_, b_ in fevs]
         eager_ms = e0.elapsed_time(e1) / dw.steps
-        # the same steps with the append as its own launch (flux_kv_write), for comparison
         n_sep = min(8, dw.steps)
         e0.record()
         for s in range(n_sep):
@@ -895,9 +972,14 @@ def run_flux(args, rank, world, dev_index):
         dec_gbs = whole_job_rate(dw.bytes_per_step, world, dec_ms, 1e9)
         fa_dec_avg = statistics.mean(fa_dec_ms)
         fa_dec_gbs = dw.bytes_fa / (fa_dec_avg * 1e-3) / 1e9
+        roof_dec = roofline_entry(fa_dec_gbs, peaks, peak_src, "hbm",
+                                  "decode_kernel<128> (FA layer, incl. its append)",
+                                  recorded_traffic("decode_fa_B16_S131072"), dw.bytes_fa,
+                                  "K+V bytes of every cached token, B 16 x (131072 + step) tokens")
         dec = {
             "workload": "qwen3-4b-36L-routed-decode: B 16, KV 131072+step, 18 FA (full cache) / "
-                        f"18 SA (ring of sink 1 + 16 blocks), fused append + decode per layer, {dw.steps} steps",
+                        f"18 SA (ring of sink 1 + 16 blocks), fused append + decode per layer, "
+                        f"{dw.steps} steps",
             "kv_resident_gb": round(dw.kv_gb, 2),
             "value": round(dec_gbs, 1), "unit": "GB/s (KV bytes that must be read)",
             "ms_per_step": round(dec_ms, 4), "gpu_launches_per_step": dw.launches,
@@ -906,63 +988,54 @@ def run_flux(args, rank, world, dev_index):
             "eager_ms_per_step": round(eager_ms, 4),
             "separate_append_eager_ms_per_step": round(separate_ms, 4),
             "frac_of_hbm": round(dec_gbs / peaks["hbm_gbs"], 4),
+            "frac_of_spec": round(dec_gbs / SPEC_HBM_GBS, 4),
             "fa_layer": {"GB/s": round(fa_dec_gbs, 1), "ms": round(fa_dec_avg, 4),
                          "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4)},
         }
-        roof_dec = {"bound": "hbm", "achieved": round(fa_dec_gbs, 1), "peak": peaks["hbm_gbs"],
-                    "unit": "GB/s", "frac": round(fa_dec_gbs / peaks["hbm_gbs"], 4),
-                    "traffic": recorded_traffic("decode_fa_B16_S131072"),
-                    "kernel": "decode_kernel<128> (FA layer, incl. its append)"}
-        dec["roofline"] = roof_dec
         dec["routing_granularity"] = dw.granularity(8)
         dec["sa_layer"] = dw.sa_layer(10)
         ctx.check()
         del dw.graph
         del dw
     torch.cuda.empty_cache()
-    extended = {}
     if not args.no_extended and world == 1:
-        from sparse_attention_flux_b200 import synth as _s
-        extended["prefill_36_layers"] = prefill_36_layers(ctx, dev, _s.seed_for(2) + 1000 * rank)
-        extended["llama_3_1_8b"] = llama_sweep(ctx, dev, _s.seed_for(4) + 1000 * rank)
+        extra["llama_3_1_8b"] = llama_sweep(ctx, dev, rank, peaks["hbm_gbs"])
     ctx.close()
 
     line = {
-        "metric": "routed-attn prefill TFLOP/s & decode KV GB/s at 1 B200; % of roofline",
+        "metric": METRIC,
         "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": bench_config(world),
-        "roofline": {"bound": "tensor", "achieved": round(fa_tflops, 1), "peak": peak_t,
-                     "unit": "TFLOP/s", "frac": round(fa_tflops / peak_t, 4),
-                     "traffic": recorded_traffic("prefill_fa_T32768"),
-                     "kernel": "prefill_kernel<128> (FA layer)",
-                     "peak_source": f"{peak_src} bf16_tflops (burst)",
-                     "frac_of_sustained": round(fa_tflops / peak_sus, 4)},
-        "sa_prefill": {"TFLOP/s": round(sa_tflops, 1), "ms": round(sa_avg, 4),
-                       "frac": round(sa_tflops / peak_t, 4)},
-        "fa_prefill": {"TFLOP/s": round(fa_tflops, 1), "ms": round(fa_avg, 4)},
-        "soft_prefill": soft_line,
-        **({"dynamic_sa": dyn_line} if dyn_line else {}),
-        "router": {"step_router_us": round(router_us, 2), "router_36_layers_us": round(router36_us, 2),
-                   "per_layer_us_36": round(router36_us / 36, 3),
-                   "context": "pages: 0.20 ms per layer (hardware not stated)"},
+        "roofline": roofline_entry(fa_tflops, peaks, peak_src, "tensor",
+                                   "prefill_kernel<128> (FA layer of the routed step)",
+                                   recorded_traffic("prefill_fa_T65536"), wl_flops_fa(),
+                                   "4 d FLOPs per causal (query, key) pair per query head; "
+                                   f"algorithmic bytes {fa_bytes} (Q, K, V read once, O written)",
+                                   long_step=True),
+        "roofline_sa_prefill": roofline_entry(sa_tflops, peaks, peak_src, "tensor",
+                                              "prefill_kernel<128> (SA layer of the routed step)",
+                                              recorded_traffic("prefill_sa_T65536"),
+                                              wl_flops_sa(),
+                                              "4 d FLOPs per computed (query, key) pair per "
+                                              "query head (sink 1 + window 16 blocks of 128)",
+                                              long_step=True),
+        "roofline_decode": roof_dec,
+        "prefill_step": step_line,
         "decode": dec,
-        **extended,
+        **extra,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
-                "how": "pinned host -> device copy of Q/K/V/hidden, router + index + FA + SA "
-                       "layers, device -> host copy of both outputs, every step; copies of "
-                       "steps k+1 / k-1 overlap step k's compute on separate streams; timed "
-                       "over K steps from the first upload to the last download (pipeline "
-                       "fill and drain included)",
+                "how": "pinned host -> device copy of the router's hidden states and of every "
+                       "layer's Q/K/V, the router + index + 36 layers, device -> host copy of "
+                       "every layer's output, every step; layer n's prefill overlaps layer "
+                       "n+1's upload and layer n-1's download on separate streams; timed over "
+                       "K steps from the first upload to the last download",
                 "steps": e2e_steps,
-                "serial_ms_per_step": round(e2e_serial_ms, 4),
                 "copy_floor_ms_per_step": round(copy_floor, 4),
-                "copy_floor_note": "the step's upload and download alone, concurrently on two "
-                                   "streams, on this machine; e2e ms / this = the pipeline's "
-                                   "overhead over the PCIe floor",
-                "serial_value": round(e2e_serial_value, 2)},
+                "copy_floor_note": "the step's uploads and downloads alone, concurrently on two "
+                                   "streams, on this machine: the PCIe floor of the e2e step"},
         "gpu_launches": launches,
         "clocks": clocks,
         "context": "pages: up to 2.8x prefill / 2.0x decode speedup vs FA baseline, hardware not "
@@ -971,25 +1044,37 @@ def run_flux(args, rank, world, dev_index):
     return line
 
 
+def wl_flops_fa():
+    return 4.0 * D * causal_pairs_fa(T_STEP) * HQ
+
+
+def wl_flops_sa():
+    return 4.0 * D * pairs_sa(T_STEP, BLOCK, SINK, WIN) * HQ
+
+
+METRIC = "routed-attn prefill TFLOP/s & decode KV GB/s at 1 B200; % of roofline"
+
+
 def bench_config(world: int) -> dict:
     """The workload both arms (this library and the oracle) report."""
-    return {"workload": "qwen3-4b-layer-routed-prefill: B 1, T 32768, Hq 32, Hkv 8, d 128, "
-                        "needles; router 32768x2560 -> MLP 5120-512-2 (layer0 FA, layer1 SA); "
-                        "SA block 128, sink 1, window 16",
-            "l2": "inputs larger than L2 (640 MB prefill, 17 GB decode KV); no flush",
+    return {"workload": "qwen3-4b-36L-routed-prefill: B 1, T 65536, Hq 32, Hkv 8, d 128, 36 "
+                        "layers each with its own Q/K/V (needles planted); router 65536x2560 -> "
+                        "MLP 5120-512-36 (18 FA / 18 SA); SA block 128, sink 1, window 16",
+            "l2": "inputs larger than L2 (27 GB of per-layer Q/K/V for prefill, 17 GB of decode "
+                  "KV); no flush",
             "parallelism": f"replicas x{world} (no exchange)"}
 
 
 class OracleSample:
-    """The oracle, as it stands, on bounded samples of the bench's prefill layer:
-    uniformly drawn query rows, FA rows for half of a sample's time, then SA rows.
-    FLOPs are counted like the GPU's (4 d per visible pair)."""
+    """The oracle, as it stands, on bounded samples of one layer of the routed prefill
+    step (T 65536, needles): uniformly drawn query rows, FA rows for half of a sample's
+    time, then SA rows.  FLOPs are counted like the GPU's (4 d per visible pair)."""
 
-    def __init__(self):
+    def __init__(self, T=T_STEP):
         import oracle
         from sparse_attention_flux_b200 import synth
-        self.oracle = oracle
-        seed = synth.seed_for(1)
+        self.oracle, self.T = oracle, T
+        seed = synth.seed_for(2)
         self.q, self.k, self.v = synth.attention_inputs(1, T, HQ, HKV, D, seed)
         synth.plant_needles_np(self.q, self.k, seed)
         self.scale = 1.0 / math.sqrt(D)
@@ -1000,6 +1085,7 @@ class OracleSample:
     def run(self, seconds):
         """One bounded sample: (visible pairs, seconds taken, rows)."""
         pairs, used, n_rows = 0, 0.0, 0
+        T = self.T
         for sparse in (False, True):
             t0 = time.perf_counter()
             while time.perf_counter() - t0 < seconds / 2:
@@ -1022,7 +1108,7 @@ class OracleSample:
 
 
 def cpu_baseline(seconds_budget=15.0, threads=None, sampler=None):
-    """The oracle on one bounded sample of the same prefill workload (all host cores,
+    """The oracle on one bounded sample of the prefill step's workload (all host cores,
     or `threads` of them)."""
     sampler = sampler or OracleSample()
     oracle = sampler.oracle
@@ -1035,8 +1121,45 @@ def cpu_baseline(seconds_budget=15.0, threads=None, sampler=None):
         oracle.set_num_threads(all_threads)
     return {"value": 4.0 * D * pairs / used / 1e12, "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle",
-            "sample": f"{n_rows} uniformly sampled query rows (half FA, half SA) of the T=32768 "
-                      f"layer, {used:.1f} s; FLOPs counted like the GPU's (4 d per visible pair)"}
+            "sample": f"{n_rows} uniformly sampled query rows (half of the time FA rows, half SA "
+                      f"rows) of one T=65536 layer of the routed step, {used:.1f} s; FLOPs "
+                      f"counted like the GPU's (4 d per visible pair)"}
+
+
+def cpu_baseline_decode(threads=None):
+    """The oracle on one sequence of the 36-layer decode workload (KV 131072 + 1 tokens,
+    Hq 32, Hkv 8, d 128): one FA-layer decode and one SA-layer decode (sink 1 + 16 blocks),
+    extrapolated to the step (16 sequences x (18 FA + 18 SA layers)); GB/s over the KV
+    bytes that must be read, like the GPU's figure."""
+    import oracle
+    from sparse_attention_flux_b200 import synth
+    s = DEC_S + 1
+    q, kc, vc = synth.decode_inputs(1, s, HQ, HKV, D, synth.seed_for(3))
+    sl = np.array([s], np.int32)
+    scale = 1.0 / math.sqrt(D)
+    if threads is not None:
+        all_threads = oracle.num_threads()
+        oracle.set_num_threads(threads)
+    cores = oracle.num_threads()
+    t0 = time.perf_counter()
+    oracle.attn_decode(q, kc, vc, sl, scale, 1, SINK, WIN, BLOCK)
+    t_fa = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    reps = 20
+    for _ in range(reps):
+        oracle.attn_decode(q, kc, vc, sl, scale, 0, SINK, WIN, BLOCK)
+    t_sa = (time.perf_counter() - t0) / reps
+    if threads is not None:
+        oracle.set_num_threads(all_threads)
+    kv_row = HKV * D * 2 * 2
+    step_s = DEC_B * (DEC_LAYERS // 2) * (t_fa + t_sa)
+    step_bytes = DEC_B * (DEC_LAYERS // 2) * (s + sa_decode_tokens(s, BLOCK, SINK, WIN)) * kv_row
+    return {"value": step_bytes / step_s / 1e9, "unit": "GB/s (KV bytes that must be read)",
+            "cores": cores, "kind": "oracle",
+            "ms_per_step_extrapolated": round(step_s * 1e3, 1),
+            "sample": f"one sequence at KV {s}: FA-layer decode {t_fa * 1e3:.1f} ms, SA-layer "
+                      f"decode {t_sa * 1e3:.2f} ms (mean of {reps}); step time extrapolated to "
+                      f"16 sequences x 18 FA + 18 SA layers"}
 
 
 def run_reference(args, world):
@@ -1054,9 +1177,10 @@ def run_reference(args, world):
         pairs, used, rows = pairs + p, used + u, rows + n
     value = 4.0 * D * pairs / used / 1e12
     sample = (f"{args.steps} steps of {per_step:.2f} s each ({args.warmup} more untimed): "
-              f"{rows} uniformly sampled query rows of the T=32768 layer (half of each step FA "
-              f"rows, half SA rows); FLOPs counted like the GPU's (4 d per visible pair)")
-    return {"metric": "routed-attn prefill TFLOP/s & decode KV GB/s at 1 B200; % of roofline",
+              f"{rows} uniformly sampled query rows of one T=65536 layer of the routed step "
+              f"(half of each step FA rows, half SA rows); FLOPs counted like the GPU's (4 d per "
+              f"visible pair)")
+    return {"metric": METRIC,
             "impl": "reference", "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": used / max(1, args.steps) * 1e3, "higher_is_better": True,
@@ -1078,7 +1202,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-extended", action="store_true",
-                    help="skip the 36-layer T 65536 prefill and the Llama-3.1-8B sweep")
+                    help="skip the T 32768 layer pair, soft blend, dynamic SA and Llama-3.1-8B runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
@@ -1112,6 +1236,11 @@ def main():
             one = cpu_baseline(4.0, threads=1, sampler=sampler)
             line["cpu_baseline"]["single_thread"] = {"value": one["value"], "cores": 1,
                                                      "sample": one["sample"]}
+            del sampler
+            if line.get("decode"):
+                dcb = cpu_baseline_decode()
+                dcb["single_thread"] = cpu_baseline_decode(threads=1)
+                line["decode"]["cpu_baseline"] = dcb
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

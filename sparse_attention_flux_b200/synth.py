@@ -90,11 +90,28 @@ def plant_needles_np(q: np.ndarray, k: np.ndarray, seed: int, n_needles: int = 1
     return needles
 
 
-def router_inputs(T: int, Hd: int, H1: int, L: int, seed: int, coin_bias: float | None = None):
+def plant_needles_torch(q, k, seed: int, n_needles: int = 16, factor: float = 3.0):
+    """plant_needles_np for device tensors (bf16 [B,T,Hq,d] / [B,T,Hkv,d]): the same
+    positions; key := factor * q row, multiplied in fp32 and rounded to bf16 (nearest
+    even), as the host version does.  In place."""
+    import torch
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    needles = needle_positions(T, Hkv, Hq // Hkv, seed, n_needles)
+    for b in range(B):
+        for g, (h, r, pos) in enumerate(needles):
+            row = (q[b, r, h].float() * factor).to(torch.bfloat16)
+            k[b, torch.from_numpy(pos).to(k.device), g] = row
+    return needles
+
+
+def router_inputs(T: int, Hd: int, H1: int, L: int, seed: int, coin_bias: float | None = None,
+                  n_positive: int | None = None):
     """(hidden bits [T,Hd], W1 [H1,2Hd], b1 [H1], W2 [L,H1], b2 [L]) with fp32 weights.
 
     coin_bias=None draws b2 ~ N(0, 0.1); otherwise b2 = +-coin_bias from a
-    seeded fair coin per layer.
+    seeded fair coin per layer, or, with n_positive given, +coin_bias on exactly
+    n_positive layers chosen by a seeded permutation and -coin_bias on the rest.
     """
     hidden = normal_bf16_bits((T, Hd), seed)
     r = rng(seed + 11)
@@ -105,6 +122,8 @@ def router_inputs(T: int, Hd: int, H1: int, L: int, seed: int, coin_bias: float 
         b2 = r.standard_normal(L, dtype=np.float32) * np.float32(0.1)
     else:
         coins = r.integers(0, 2, size=L)
+        if n_positive is not None:
+            coins = (rng(seed + 12).permutation(L) < n_positive).astype(np.int64)
         b2 = np.where(coins == 1, np.float32(coin_bias), np.float32(-coin_bias)).astype(np.float32)
     return hidden, W1, b1, W2, b2
 

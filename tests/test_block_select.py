@@ -1,10 +1,16 @@
 """Dynamic SA block selection on the GPU against the oracle.
 
-The scores (fp32 on the GPU, fp64 in the oracle) are compared element by element;
-the mask is an integer decided from fp32 scores, so the oracle's selection is run
-on the GPU's own scores and must match bit for bit.  The selected mask then drives
-the CSR builder and SA prefill, compared with the oracle's attention under the same
-mask."""
+Scores: the GPU's fp32 scores are compared with the oracle's fp64 scores element
+by element, within a bound relative to each element (SCORE_RTOL * P + SCORE_ATOL;
+see _score_bound).  Mask: (1) the GPU mask equals the oracle's selection run on the
+GPU's own fp32 scores, bit for bit (the selection kernel against its definition);
+(2) end to end, the GPU mask equals the oracle's own pipeline (oracle scores, then
+the oracle's fp32 selection), except at candidates whose decision the score bound
+leaves open -- where the oracle's running sum before the candidate lies within the
+row's summed score bound of tau, or where two differing candidates' scores are
+within their bounds of each other -- and the tests count such bits (zero in every
+case measured).  The selected mask then drives the CSR builder and SA prefill,
+compared with the oracle's attention under the same mask."""
 import math
 
 import numpy as np
@@ -17,6 +23,76 @@ from sparse_attention_flux_b200.flux import Context
 from helpers import assert_close_attn, bits_of
 
 pytestmark = pytest.mark.gpu
+
+# Per-element score bound.  The GPU's logits are fp32 tensor-core sums of 8 d exact
+# bf16 products, turned into per-key-block log-sum-exps with ex2/lg2 (about 2^-22
+# relative each); a share P = 2^(lse_j - lse_total) then carries a relative error
+# of a few logit roundings.  Measured on B200 over every case below and the full
+# sizes: at most 8.2e-6 relative (6.1e-7 absolute).  The bound leaves a factor of
+# about 6 above that, and an absolute floor for shares near fp32's underflow.
+SCORE_RTOL = 5e-5
+SCORE_ATOL = 1e-7
+
+
+def _score_bound(P):
+    return SCORE_ATOL + SCORE_RTOL * np.abs(P)
+
+
+def _assert_scores_within_bound(score_row, P_row, what):
+    err = np.abs(score_row.astype(np.float64) - P_row)
+    bound = _score_bound(P_row)
+    worst = int(np.argmax(err - bound))
+    assert np.all(err <= bound), (f"{what}: score error {err[worst]:.3e} at key block {worst} "
+                                  f"(oracle {P_row[worst]:.6e}, bound {bound[worst]:.3e})")
+
+
+def _open_decisions(p, tau, sink, i):
+    """For query block i with oracle scores p[0..i] (fp64): the oracle's order of the
+    candidates (score descending, block ascending, as fp32 -- the selection's own
+    precision) and, per candidate, the fp32 running sum before it."""
+    p32 = p[:i + 1].astype(np.float32)
+    forced = [j for j in range(i + 1) if j < sink or j == i]
+    cand = sorted((j for j in range(i + 1) if not (j < sink or j == i)),
+                  key=lambda j: (-p32[j], j))
+    cum = np.float32(0)
+    for j in forced:
+        cum = np.float32(cum + p32[j])
+    before = {}
+    for j in cand:
+        before[j] = float(cum)
+        cum = np.float32(cum + p32[j])
+    return before
+
+
+def _mask_vs_oracle_pipeline(mask, P_rows, rows, tau, sink, what):
+    """The GPU mask against the oracle's own pipeline (oracle scores -> oracle
+    selection) on the listed query blocks.  A differing bit is allowed only where
+    the decision is open under the score bound: the oracle's running sum before
+    that candidate within the row's summed bound of tau, or another differing
+    candidate whose score is within both bounds of this one.  Returns how many
+    such bits there were."""
+    nb = mask.shape[1]
+    full = np.zeros((nb, nb), np.float64)
+    for n, i in enumerate(rows):
+        full[i] = P_rows[n]
+    m_or = oracle.select_blocks(full, tau, sink)
+    open_bits = 0
+    for n, i in enumerate(rows):
+        diff = np.nonzero(m_or[i] != mask[i])[0]
+        if diff.size == 0:
+            continue
+        p = P_rows[n]
+        e = _score_bound(p)
+        row_bound = float(e[:i + 1].sum())
+        before = _open_decisions(p, tau, sink, i)
+        for j in diff:
+            near_tau = j in before and abs(before[j] - tau) <= row_bound
+            near_tie = any(j2 != j and abs(p[j] - p[j2]) <= e[j] + e[j2] for j2 in diff)
+            assert near_tau or near_tie, (f"{what}: query block {i}, key block {j}: GPU mask "
+                                          f"{mask[i, j]} vs oracle {m_or[i, j]} with the decision "
+                                          f"not open under the score bound")
+            open_bits += 1
+    return open_bits
 
 
 @pytest.fixture(scope="module")
@@ -59,12 +135,17 @@ def test_scores_and_mask_match_oracle(ctx, case):
     P = oracle.block_scores(q, k, 128, stride, 1 / math.sqrt(d))
     nb = P.shape[0]
     lower = np.tril(np.ones((nb, nb), bool))
-    err = np.abs(score.astype(np.float64) - P)
-    assert err[lower].max() <= 5e-5 + 1e-3 * P[lower].max(), f"{case}: score error {err.max()}"
+    for i in range(nb):
+        _assert_scores_within_bound(score[i, :i + 1], P[i, :i + 1], f"{case} row {i}")
     assert np.all(score[~lower] == 0)
-    np.testing.assert_allclose(score.astype(np.float64).sum(axis=1), 1.0, atol=1e-4)
-    # the integer decision, taken by the oracle on the GPU's fp32 scores
+    # the row sums follow from the per-element bound
+    np.testing.assert_allclose(score.astype(np.float64).sum(axis=1), 1.0,
+                               atol=SCORE_RTOL + nb * SCORE_ATOL)
+    # the selection kernel against its definition, on the GPU's own fp32 scores
     np.testing.assert_array_equal(mask, oracle.select_blocks(score, tau, sink), err_msg=str(case))
+    # end to end against the oracle's own scores and selection
+    open_bits = _mask_vs_oracle_pipeline(mask, P, list(range(nb)), tau, sink, str(case))
+    print(f"{case}: {open_bits} mask bits differ from the oracle pipeline (all open decisions)")
 
 
 def test_planted_block_is_selected(ctx):
@@ -112,18 +193,23 @@ def test_deterministic(ctx):
 
 
 def _sampled_rows_check(score, mask, q, k, d, rows, tau, sink, what):
-    """Sampled score rows against the oracle, then properties of the whole GPU matrix:
-    rows sum to 1, nothing above the diagonal, and the mask is the oracle's selection
-    on the GPU's fp32 scores, bit for bit."""
+    """Sampled score rows against the oracle within the per-element bound; properties
+    of the whole GPU matrix (rows sum to 1, nothing above the diagonal, the mask is the
+    oracle's selection on the GPU's fp32 scores, bit for bit); and the sampled rows of
+    the mask against the oracle's own pipeline."""
     nb = score.shape[0]
     P = oracle.block_scores_rows(q, k, 128, 8, 1 / math.sqrt(d), rows)
     for n, i in enumerate(rows):
-        err = np.abs(score[i, :i + 1].astype(np.float64) - P[n, :i + 1])
-        assert err.max() <= 5e-5 + 1e-3 * P[n, :i + 1].max(), f"{what}: row {i} error {err.max()}"
+        _assert_scores_within_bound(score[i, :i + 1], P[n, :i + 1], f"{what} row {i}")
     upper = np.triu(np.ones((nb, nb), bool), 1)
     assert np.all(score[upper] == 0) and np.all(mask[upper] == 0)
-    np.testing.assert_allclose(score.astype(np.float64).sum(axis=1), 1.0, atol=1e-4)
+    # the row sums follow from the per-element bound
+    np.testing.assert_allclose(score.astype(np.float64).sum(axis=1), 1.0,
+                               atol=SCORE_RTOL + nb * SCORE_ATOL)
     np.testing.assert_array_equal(mask, oracle.select_blocks(score, tau, sink), err_msg=what)
+    open_bits = _mask_vs_oracle_pipeline(mask, P, rows, tau, sink, what)
+    print(f"{what}: {open_bits} mask bits of the sampled rows differ from the oracle pipeline "
+          f"(all open decisions)")
 
 
 def test_qwen3_4b_layer_sampled_rows(ctx):
