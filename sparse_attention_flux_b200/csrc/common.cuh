@@ -43,6 +43,20 @@ __device__ __forceinline__ long long globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while the
+// previous kernel in the stream is still running.  griddep_wait() blocks until
+// that kernel has completed and its memory writes are visible; nothing the
+// previous kernel may have written can be read (or overwritten) before it.
+// griddep_launch_dependents() lets the next such kernel be launched once every
+// CTA of this grid has called it (or exited).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

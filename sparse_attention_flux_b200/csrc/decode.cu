@@ -148,6 +148,14 @@ __global__ void __launch_bounds__(kThreads, 2)
   // leaves idle (launched for the FA range) only exit after them.
   const int i = blockIdx.z, g = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Launched with programmatic stream serialisation: the next decode launch may
+  // be dispatched as soon as every CTA of this one has started, and this CTA
+  // starts before the previous kernel has finished.  Everything below reads or
+  // writes memory that kernel may touch (routing bits, lengths, q, the cache,
+  // the split partials and merge tickets of a shared workspace), so it waits
+  // for that kernel first; what overlaps is the launch and the CTA dispatch.
+  griddep_launch_dependents();
+  griddep_wait();
   const int G = a.Hq / a.Hkv;   // 1..kMaxGroup, checked on the host
   // Per-head routing: the group reads the FA range if any of its heads is FA;
   // its SA heads then mask every token outside the sink + window blocks.
@@ -429,9 +437,19 @@ cudaError_t launch_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeL
                      cudaStream_t stream) {
   const int smem = DSmem<D>::ALLOC;
   cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  const dim3 grid(p.Hkv, p.B, p.nsplit);
-  decode_kernel<D><<<grid, kThreads, smem, stream>>>(tk, tv, p);
-  return cudaGetLastError();
+  // Programmatic stream serialisation: consecutive decode launches (one per
+  // layer) overlap the next launch's dispatch with this one's tail.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.Hkv, p.B, p.nsplit);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<D>, tk, tv, p);
 }
 
 }  // namespace
