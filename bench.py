@@ -572,8 +572,10 @@ class DecodeWorkload:
 
     def sa_layer(self, reps):
         """One SA layer's decode over its compact ring (B 16, the last step's length), timed
-        launch by launch: back to back (ring partly L2-resident: 143 MB of K+V against a
-        126 MB L2) and with a 256 MB write between launches (cold L2)."""
+        launch by launch with CUDA events around each eager launch: back to back (ring
+        partly L2-resident: 143 MB of K+V against a 126 MB L2) and with a 256 MB write
+        between launches (cold L2); and 40 launches replayed from a CUDA graph (the
+        GPU-side cost per layer, without the host's per-call submission)."""
         import torch
         layer = min(self.rings)
         kr, vr = self.rings[layer]
@@ -596,8 +598,32 @@ class DecodeWorkload:
             torch.cuda.synchronize()
             us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
             out[name] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1)}
+        # Back to back from a CUDA graph of 40 launches: the GPU-side cost of a layer
+        # with no host submission in it (each launch's dispatch overlaps the previous
+        # one's tail: programmatic dependent launch).
+        n_graph = 40
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(self.dev)
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=cs):
+            for _ in range(n_graph):
+                fn()
+        torch.cuda.current_stream().wait_stream(cs)
+        g.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) / n_graph * 1e3)
+        us = statistics.median(ts)
+        out["graph_back_to_back"] = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
+                                     "launches": n_graph}
         out["kv_bytes"] = byts
-        del flush
+        del g, flush
         return out
 
     def capture(self):
@@ -724,9 +750,10 @@ def llama_sweep(ctx, dev, rank, hbm_gbs):
     32-layer step (mask + CSR + 32 launches reading their bits on the device) measured
     once per SA fraction 0/25/50/75/100 % at W 16 and at 50 % for W 8 and 32, after one
     warm-up step; per-layer CUDA events give the FA and SA layer rates inside it.
-    decode, B 4, S 131072: the whole 32-layer step measured at SA fractions
-    0/25/50/75/100 % (W 16) and at 50 % for W 8 and 32; every layer has its own full
-    cache (2.15 GB; 69 GB in all), so no layer's window is left in L2 by another's."""
+    decode, B 4, S 131072: the whole 32-layer step, replayed from a CUDA graph (and launched
+    eagerly, for comparison), at SA fractions 0/25/50/75/100 % (W 16) and at 50 % for W 8
+    and 32; every layer has its own full cache (2.15 GB; 69 GB in all), so no layer's
+    window is left in L2 by another's."""
     import torch
     from sparse_attention_flux_b200 import synth
     L, T3, B4, S4 = 32, 131072, 4, 131072
@@ -804,15 +831,31 @@ def llama_sweep(ctx, dev, rank, hbm_gbs):
         b.synchronize()
         return a.elapsed_time(b) / n
 
+    def graph_timed(fn, n):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(dev)
+        cs.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=cs):
+            fn()
+        torch.cuda.current_stream().wait_stream(cs)
+        ms = timed(g.replay, n)
+        del g
+        return ms
+
     dec = {}
     for pct, W in [(0, 16), (25, 16), (50, 16), (75, 16), (100, 16), (50, 8), (50, 32)]:
         n_sa = L * pct // 100
         mode_t = torch.from_numpy(synth.layer_mode_choice(L, L - n_sa, synth.seed_for(4) + pct)).to(dev)
-        ms = timed(lambda: dec_step(mode_t, W), 5)
+        eager_ms = timed(lambda: dec_step(mode_t, W), 5)
+        ms = graph_timed(lambda: dec_step(mode_t, W), 5)
         byts = B4 * ((L - n_sa) * S4 + n_sa * sa_decode_tokens(S4, BLOCK, SINK, W)) * kv_row
         dec[f"sa{pct}%_W{W}"] = {"ms_per_step": round(ms, 3),
                                  "GB/s": round(byts / (ms * 1e-3) / 1e9, 1),
-                                 "frac_of_hbm": round(byts / (ms * 1e-3) / 1e9 / hbm_gbs, 4)}
+                                 "frac_of_hbm": round(byts / (ms * 1e-3) / 1e9 / hbm_gbs, 4),
+                                 "eager_ms_per_step": round(eager_ms, 3)}
+    dec["how"] = ("the 32-layer step (one decode launch per layer, each reading its routing bit "
+                  "on the device) captured once as a CUDA graph and replayed 5 times; "
+                  "eager_ms_per_step launches the same step from the host")
     ctx.check()
     out["decode"] = dec
     del caches
