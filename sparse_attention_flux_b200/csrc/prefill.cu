@@ -535,7 +535,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t row_elem = ((static_cast<size_t>(b) * a.T + t_row) * a.Hq + h) * D;
     const bool valid = t_row < a.T;
     // One decision per warpgroup (a named barrier below needs all 128 threads).
+    // Barrier instructions are warp-aligned and lanes may have left the tile
+    // loop apart (a wait that gave up), so the warp reconverges first.
     const bool mine = n > 0 && ok && mbar_wait(&bars[B_OD], 0, a.st);
+    __syncwarp();
     const bool have_o = named_bar_and(1 + i, 128, mine);
     if (have_o && !a.blend_score) {
       // O_i / l -> bf16 rows staged in Q_i's (now free: every MMA has completed)
