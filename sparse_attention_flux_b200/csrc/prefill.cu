@@ -13,8 +13,8 @@
 //     so no MMA or softmax is spent on a tile that only one of them sees; or
 //   a row pair (odd group size, or per-head routing): rows [256u, 256u + 256)
 //     of one query head, walking the union of the two tiles' lists.
-// CTAs are ordered per sequence, in chunks of kv groups whose K/V fit in L2,
-// longest unit first within a chunk.
+// CTAs are ordered per sequence, in chunks of kv groups whose K/V fit in 48 MB
+// of L2, longest unit first within a chunk.
 //
 // Per CTA (384 threads, warp-specialised):
 //   warp 0      TMA producer (Q0, Q1 once; K/V tiles into a 2-stage ring, K
@@ -652,13 +652,15 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   a.nunit = a.head_pair ? (p.T + kBM - 1) / kBM : (p.T + 2 * kBM - 1) / (2 * kBM);
   a.nkt = (p.T + kBN - 1) / kBN;
   // As many kv groups per chunk (a divisor of Hkv) as keep their K and V
-  // within 72 MB, inside L2 beside the Q and O streams (measured: DRAM reads
-  // fall to the algorithmic bytes; 48 MB cost 1.4 %, 72 MB nothing).
+  // within 48 MB, inside L2 beside the Q and O streams, so that the CTAs in
+  // flight re-read K and V from L2 rather than DRAM (measured at T 65536 in a
+  // power-capped run of FA layers: the same time as a 72 MB chunk, which let
+  // DRAM reads reach about 1.9x the algorithmic bytes).
   {
     const long long kv_bytes = 4LL * p.T * p.d;   // K + V of one group, bf16
     a.gchunk = 1;
     for (int gcand = p.Hkv; gcand > 1; --gcand)
-      if (p.Hkv % gcand == 0 && gcand * kv_bytes <= (72LL << 20)) { a.gchunk = gcand; break; }
+      if (p.Hkv % gcand == 0 && gcand * kv_bytes <= (48LL << 20)) { a.gchunk = gcand; break; }
   }
   a.block = p.block;
   a.nqb = p.nqb;
