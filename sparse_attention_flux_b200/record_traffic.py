@@ -1,7 +1,7 @@
 """Record a kernel's measured DRAM traffic for the bench's roofline line.
 
     python -m sparse_attention_flux_b200.record_traffic KEY REPORT.ncu-rep --scale S \
-        --workload "..." --capture profiles/....md SOURCE [SOURCE ...]
+        --workload "..." --capture SUMMARY SOURCE [SOURCE ...]
 
 Reads dram__bytes_read.sum and dram__bytes_write.sum of the (single) launch in
 an ncu report (``ncu -i REPORT --page raw --csv``), multiplies their sum by S
@@ -64,7 +64,7 @@ def main() -> None:
     ap.add_argument("sources", nargs="+", help="repo-relative source files of the kernel")
     ap.add_argument("--scale", type=float, default=1.0)
     ap.add_argument("--workload", required=True)
-    ap.add_argument("--capture", required=True, help="the profiles/ summary of the capture")
+    ap.add_argument("--capture", required=True, help="the summary file of the capture")
     args = ap.parse_args()
     rd, wr = dram_bytes(args.report)
     rec = {}
