@@ -59,6 +59,7 @@ BLOCK, SINK, WIN = 128, 1, 16
 T_STEP, L_STEP = 65536, 36                 # the routed prefill step
 T_PAIR = 32768                              # the single-layer pair (extra)
 DEC_B, DEC_S, DEC_LAYERS, DEC_STEPS = 16, 131072, 36, 64
+E2E_BUFFERS = 4                             # layers' inputs/outputs in flight in the e2e step
 # Dense bf16 tensor and HBM figures of the B200 specification, beside the measured peaks.
 SPEC_TFLOPS, SPEC_HBM_GBS = 2250.0, 8000.0
 
@@ -331,8 +332,12 @@ class RoutedPrefill:
         # work).  Two pinned output buffers take the layers' outputs in turn.
         self.qkv_h = [x.cpu().pin_memory() for x in (st.q[0], st.k[0], st.v[0])]
         self.o_h = [torch.empty(st.o.shape, dtype=st.o.dtype).pin_memory() for _ in range(2)]
-        self.ins = [[torch.empty_like(x) for x in (st.q[0], st.k[0], st.v[0])] for _ in range(2)]
-        self.outs = [torch.empty_like(st.o) for _ in range(2)]
+        # Device buffers for E2E_BUFFERS layers in flight: uploads run ahead while an FA
+        # layer computes (an FA layer takes about twice a layer's upload, an SA layer a
+        # tenth of it).
+        self.ins = [[torch.empty_like(x) for x in (st.q[0], st.k[0], st.v[0])]
+                    for _ in range(E2E_BUFFERS)]
+        self.outs = [torch.empty_like(st.o) for _ in range(E2E_BUFFERS)]
         self.hid_d = torch.empty_like(self.hidden)
 
     @property
@@ -345,15 +350,17 @@ class RoutedPrefill:
 
     def e2e_pipelined(self, steps):
         """The step from pinned host memory through the public API, pipelined per layer
-        over three streams: layer n's prefill overlaps layer n+1's host->device copy of
-        Q/K/V and layer n-1's device->host copy of its output (double-buffered device
-        tensors); each step first uploads the router's hidden states.  Returns ms per
-        step, from an event before the first copy to one after the last copy back."""
+        over three streams: layer n's prefill overlaps the host->device copies of the
+        next layers' Q/K/V (up to E2E_BUFFERS - 1 ahead) and the device->host copies of
+        earlier layers' outputs; each step first uploads the router's hidden states.
+        Returns ms per step, from an event before the first copy to one after the last
+        copy back."""
         import torch
         dev, c, st = self.dev, self.ctx, self.stack
         s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
         ev = lambda: torch.cuda.Event(enable_timing=False)
-        h2d, cmp, d2h = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        nbuf = E2E_BUFFERS
+        h2d, cmp, d2h = ([ev() for _ in range(nbuf)] for _ in range(3))
         hid_done, head_done = ev(), ev()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
@@ -370,16 +377,16 @@ class RoutedPrefill:
                 self.head(self.hid_d, stream=s_cmp)
                 head_done.record(s_cmp)
             for l in range(L_STEP):
-                b = n % 2
+                b = n % nbuf
                 with torch.cuda.stream(s_in):
-                    if n >= 2:
+                    if n >= nbuf:
                         s_in.wait_event(cmp[b])
                     for dst, x in zip(self.ins[b], self.qkv_h):
                         dst.copy_(x, non_blocking=True)
                     h2d[b].record(s_in)
                 with torch.cuda.stream(s_cmp):
                     s_cmp.wait_event(h2d[b])
-                    if n >= 2:
+                    if n >= nbuf:
                         s_cmp.wait_event(d2h[b])
                     q, kk, v = self.ins[b]
                     c.attn_prefill(q, kk, v, self.outs[b], st.scale, layer_mode=self.mode,
@@ -388,7 +395,7 @@ class RoutedPrefill:
                     cmp[b].record(s_cmp)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(cmp[b])
-                    self.o_h[b].copy_(self.outs[b], non_blocking=True)
+                    self.o_h[n % 2].copy_(self.outs[b], non_blocking=True)
                     d2h[b].record(s_out)
                 n += 1
         s_out.wait_stream(s_in)
@@ -411,11 +418,11 @@ class RoutedPrefill:
             with torch.cuda.stream(s_in):
                 self.hid_d.copy_(self.hidden_h, non_blocking=True)
                 for l in range(L_STEP):
-                    for dst, x in zip(self.ins[l % 2], self.qkv_h):
+                    for dst, x in zip(self.ins[l % E2E_BUFFERS], self.qkv_h):
                         dst.copy_(x, non_blocking=True)
             with torch.cuda.stream(s_out):
                 for l in range(L_STEP):
-                    self.o_h[l % 2].copy_(self.outs[l % 2], non_blocking=True)
+                    self.o_h[l % 2].copy_(self.outs[l % E2E_BUFFERS], non_blocking=True)
         s_in.wait_stream(s_out)
         b.record(s_in)
         b.synchronize()
@@ -1095,9 +1102,10 @@ def run_flux(args, rank, world, dev_index):
                 "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                 "how": "pinned host -> device copy of the router's hidden states and of every "
                        "layer's Q/K/V, the router + index + 36 layers, device -> host copy of "
-                       "every layer's output, every step; layer n's prefill overlaps layer "
-                       "n+1's upload and layer n-1's download on separate streams; timed over "
-                       "K steps from the first upload to the last download",
+                       "every layer's output, every step; layer n's prefill overlaps the "
+                       "uploads of up to 3 later layers and the downloads of earlier ones on "
+                       "separate streams (4 layers' buffers in flight); timed over K steps "
+                       "from the first upload to the last download",
                 "steps": e2e_steps,
                 "copy_floor_ms_per_step": round(copy_floor, 4),
                 "copy_floor_note": "the step's uploads and downloads alone, concurrently on two "
