@@ -59,7 +59,7 @@ BLOCK, SINK, WIN = 128, 1, 16
 T_STEP, L_STEP = 65536, 36                 # the routed prefill step
 T_PAIR = 32768                              # the single-layer pair (extra)
 DEC_B, DEC_S, DEC_LAYERS, DEC_STEPS = 16, 131072, 36, 64
-E2E_BUFFERS = 4                             # layers' inputs/outputs in flight in the e2e step
+E2E_BUFFERS = 8                             # layers' inputs/outputs in flight in the e2e step
 # Dense bf16 tensor and HBM figures of the B200 specification, beside the measured peaks.
 SPEC_TFLOPS, SPEC_HBM_GBS = 2250.0, 8000.0
 
@@ -1103,8 +1103,8 @@ def run_flux(args, rank, world, dev_index):
                 "how": "pinned host -> device copy of the router's hidden states and of every "
                        "layer's Q/K/V, the router + index + 36 layers, device -> host copy of "
                        "every layer's output, every step; layer n's prefill overlaps the "
-                       "uploads of up to 3 later layers and the downloads of earlier ones on "
-                       "separate streams (4 layers' buffers in flight); timed over K steps "
+                       "uploads of up to 7 later layers and the downloads of earlier ones on "
+                       "separate streams (8 layers' buffers in flight); timed over K steps "
                        "from the first upload to the last download",
                 "steps": e2e_steps,
                 "copy_floor_ms_per_step": round(copy_floor, 4),
