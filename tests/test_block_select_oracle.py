@@ -7,6 +7,8 @@ parity against the pages is unpinned; these tests pin the oracle to the
 definition itself by routes that share none of its code: the full T x T score
 matrix from a library matmul with the antidiagonals indexed explicitly, closed
 forms, invariants and hand-enumerated selections."""
+import math
+
 import numpy as np
 import pytest
 
@@ -192,3 +194,52 @@ def test_sampled_rows_reject_out_of_range():
         oracle.block_scores_rows(q, k, 128, 8, 0.25, [2])
     with pytest.raises(ValueError):
         oracle.block_scores_rows(q, k, 128, 8, 0.25, [-1])
+
+
+def _selection_boundary_case():
+    """Oracle scores of a small layer and a tau that lies just above the running sum
+    before one candidate of the last query block, so that any score error larger than
+    the bound moves that decision."""
+    q, k, _ = synth.attention_inputs(1, 2048, 2, 1, 64, seed=71)
+    P = oracle.block_scores(q, k, 128, 8, 1 / math.sqrt(64))
+    nb = P.shape[0]
+    i = nb - 1
+    p32 = P[i, :i + 1].astype(np.float32)
+    forced = [0, i]
+    cand = sorted((j for j in range(1, i)), key=lambda j: (-p32[j], j))
+    cum = np.float32(0)
+    for j in forced:
+        cum = np.float32(cum + p32[j])
+    for j in cand[:4]:
+        cum = np.float32(cum + p32[j])
+    # the fifth candidate is taken iff the running sum (cum) is below tau
+    tau = float(np.float32(cum) + np.float32(2e-4))
+    return P, tau
+
+
+def test_mask_check_rejects_a_biased_selection():
+    """The parity check of the GPU selector, pinned by planting a mistake in the oracle:
+    scores with a systematic relative bias 20x the stated bound flip a selection near
+    tau; the score check and the mask check against the oracle's own pipeline both
+    reject them, while scores within the bound pass both."""
+    from helpers import (SCORE_RTOL, assert_scores_within_bound, mask_vs_oracle_pipeline)
+    P, tau = _selection_boundary_case()
+    nb = P.shape[0]
+    i = nb - 1
+    rows = [i]
+    # a bias that raises the forced and first candidates' shares: the fifth candidate drops
+    biased = P.copy()
+    biased[i, :i + 1] *= 1.0 + 20 * SCORE_RTOL
+    m_biased = oracle.select_blocks(biased, tau, 1)
+    m_exact = oracle.select_blocks(P, tau, 1)
+    assert (m_biased[i] != m_exact[i]).any(), "the planted bias must change the selection"
+    with pytest.raises(AssertionError):
+        assert_scores_within_bound(biased[i, :i + 1].astype(np.float32), P[i, :i + 1], "biased")
+    with pytest.raises(AssertionError):
+        mask_vs_oracle_pipeline(m_biased, P[rows], rows, tau, 1, "biased")
+    # within the bound: both checks pass and no mask bit differs
+    small = P.copy()
+    small[i, :i + 1] *= 1.0 + 0.1 * SCORE_RTOL
+    assert_scores_within_bound(small[i, :i + 1].astype(np.float32), P[i, :i + 1], "small")
+    m_small = oracle.select_blocks(small, tau, 1)
+    assert mask_vs_oracle_pipeline(m_small, P[rows], rows, tau, 1, "small") == 0
