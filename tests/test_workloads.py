@@ -54,32 +54,37 @@ def _check_rows(o, lse, q, k, v, rows, block_mask, block, what):
 
 
 def test_qwen3_4b_36_layer_routed_prefill(ctx):
-    """Router on hidden 65536 x 2560 (MLP 5120 -> 512 -> 36), then one FA-routed and one
-    SA-routed layer at T 65536 (block 128, sink 1, window 16), each reading its bit on the
-    device; sampled rows against the oracle with the oracle's own routing."""
+    """The bench's routed step at T 65536 with the bench's own inputs: the router on hidden
+    65536 x 2560 (MLP 5120 -> 512 -> 36, b2 = +4 on 18 seeded layers and -4 on the rest),
+    bit-exact against the oracle's routing (18 FA / 18 SA); then the first FA-routed and the
+    first SA-routed layer, each with its own Q/K/V and planted needles as the bench draws
+    them (block 128, sink 1, window 16), each reading its bit on the device; sampled rows
+    and every needle row against the oracle."""
     T, dev = 65536, ctx.device
     hidden, W1, b1, W2, b2 = synth.router_inputs(T, 2560, 512, 36, synth.seed_for(2),
-                                                 coin_bias=2.0)
-    mode_o, _, _ = oracle.route(hidden, W1, b1, W2, b2, 0.5)
+                                                 coin_bias=4.0, n_positive=18)
+    mode_o, z, _ = oracle.route(hidden, W1, b1, W2, b2, 0.5)
     lm = torch.empty(36, dtype=torch.uint8, device=dev)
     ctx.route(synth.torch_from_bits(hidden).to(dev),
               *(torch.from_numpy(x).to(dev) for x in (W1, b1, W2, b2)), 0.5, lm)
     assert np.array_equal(lm.cpu().numpy(), mode_o)
+    assert int(mode_o.sum()) == 18 and np.abs(z).min() > 1.0
     del hidden
     rp, col = _index(ctx, T, 128, 1, 16)
     nb = T // 128
     mask = oracle.streaming_mask(nb, nb, 1, 16)
     for layer in (int(np.argmax(mode_o == 1)), int(np.argmax(mode_o == 0))):
-        seed = synth.seed_for(2, layer)
-        q = synth.torch_normal_bf16((1, T, HQ, D), seed, dev)
-        k = synth.torch_normal_bf16((1, T, HKV, D), seed + 1, dev)
-        v = synth.torch_normal_bf16((1, T, HKV, D), seed + 2, dev)
+        q = synth.torch_normal_bf16((1, T, HQ, D), synth.seed_for(2, layer, 1), dev)
+        k = synth.torch_normal_bf16((1, T, HKV, D), synth.seed_for(2, layer, 2), dev)
+        v = synth.torch_normal_bf16((1, T, HKV, D), synth.seed_for(2, layer, 3), dev)
+        needles = synth.plant_needles_torch(q, k, synth.seed_for(2, layer, 0))
         o = torch.empty_like(q)
         lse = torch.empty((1, HQ, T), dtype=torch.float32, device=dev)
         ctx.attn_prefill(q, k, v, o, SCALE, layer_mode=lm, layer=layer, row_ptr=rp, col=col,
                          block=128, lse=lse)
         ctx.check()
-        rows = _rows(T, seed + 7, 10)
+        rows = _rows(T, synth.seed_for(2, layer, 7), 10)
+        rows = np.concatenate([rows, np.array([(0, h, r) for (h, r, _) in needles], np.int32)])
         _check_rows(bits_of(o), lse.cpu().numpy(), bits_of(q), bits_of(k), bits_of(v), rows,
                     None if mode_o[layer] else mask, 128, f"layer {layer} mode {mode_o[layer]}")
 
