@@ -27,6 +27,11 @@
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream) and returns an int status.  Host-side argument
  *     checks happen before any launch; on failure nothing is launched.
+ *   - Stream order holds as usual.  The decode calls and the router's second
+ *     kernel are launched with programmatic stream serialisation: their CTAs
+ *     may be dispatched while the previous kernel on the stream finishes, but
+ *     they read and write no memory until that kernel has completed and its
+ *     writes are visible, so the caller sees ordinary stream semantics.
  *   - Device-side checks (seqlens beyond capacity, CSR entries out of range,
  *     a bounded wait that ran out) set the context's device error word and
  *     zero the affected outputs; flux_ctx_check() reports it.
@@ -238,7 +243,8 @@ int flux_attn_prefill_soft(flux_ctx* ctx, const uint16_t* q, const uint16_t* k, 
  * the group (atomic ticket, no spin) merges the partials.  Partials live in
  * the ctx workspace (flux_decode_workspace_bytes).  Supported: d 64/128,
  * Hq/Hkv a whole number from 1 to 8 (else UNSUPPORTED).  Calls sharing a ctx
- * must not overlap in time. */
+ * must not overlap in time.  Consecutive decode calls on one stream (one per
+ * layer) overlap each launch's dispatch with the previous one's tail. */
 int flux_attn_decode(flux_ctx* ctx, const uint16_t* q, const uint16_t* k_cache,
                      const uint16_t* v_cache, int S_max, const int32_t* seqlens,
                      uint16_t* o, float* lse, int B, int Hq, int Hkv, int d,
