@@ -475,12 +475,24 @@ __global__ void __launch_bounds__(kSelectThreads)
     float cum = 0.f;
     for (int j = 0; j <= i; ++j)
       if (sel[j]) cum += P[j];
-    for (int t = 0; t < n2 && cum < tau; ++t) {
-      const uint64_t x = key[t];
-      if (x == ~0ull) break;
-      const int j = static_cast<int>(x & 0xffffffffu);
-      sel[j] = 1;
-      cum += P[j];
+    // The candidates in order, each taken while the running sum is below tau.
+    // A key carries its score's bits, so the loop needs one shared-memory read
+    // per candidate, issued eight at a time; the sum is the same sequential
+    // fp32 sum in the same order.
+    bool more = true;
+    for (int t0 = 0; more && t0 < n2; t0 += 8) {
+      uint64_t xs[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) xs[k] = t0 + k < n2 ? key[t0 + k] : ~0ull;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (!more || !(cum < tau) || xs[k] == ~0ull) {
+          more = false;
+          continue;
+        }
+        sel[static_cast<int>(xs[k] & 0xffffffffu)] = 1;
+        cum += __uint_as_float(~static_cast<uint32_t>(xs[k] >> 32));
+      }
     }
   }
   __syncthreads();
