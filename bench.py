@@ -28,7 +28,7 @@ step at T 131072 measured as one step per SA fraction 0/25/50/75/100 % and per
 window 8/16/32 blocks; the 32-layer decode step at B 4, S 131072); --no-extended
 skips them.
 
-Every input is seeded and synthetic; every timed input (27 GB of Q/K/V for the
+Every input is seeded and synthetic; every timed input (29 GB of Q/K/V for the
 prefill step, 17 GB of KV for decode) is larger than the 126 MB L2, so no flush is
 needed.  Multi-GPU: the units are independent (no exchange), so each rank runs its
 own replica of the step (weak scaling) and rank 0 reports the max time.
@@ -1134,7 +1134,7 @@ def bench_config(world: int) -> dict:
     return {"workload": "qwen3-4b-36L-routed-prefill: B 1, T 65536, Hq 32, Hkv 8, d 128, 36 "
                         "layers each with its own Q/K/V (needles planted); router 65536x2560 -> "
                         "MLP 5120-512-36 (18 FA / 18 SA); SA block 128, sink 1, window 16",
-            "l2": "inputs larger than L2 (27 GB of per-layer Q/K/V for prefill, 17 GB of decode "
+            "l2": "inputs larger than L2 (29 GB of per-layer Q/K/V for prefill, 17 GB of decode "
                   "KV); no flush",
             "parallelism": f"replicas x{world} (no exchange)"}
 
