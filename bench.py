@@ -271,15 +271,15 @@ class LayerStack:
         f_sa = 4.0 * D * pairs_sa(self.T, BLOCK, SINK, W) * HQ
         return sum(f_fa if m else f_sa for m in mode_h), f_fa, f_sa
 
-    def layers(self, mode, row_ptr, col, evs=None, q=None, k=None, v=None, o=None, stream=None):
+    def layers(self, mode, row_ptr, col, evs=None):
+        """Every layer's prefill launch, each reading its bit mode[l] on the device;
+        CUDA events around each launch when given."""
         c = self.ctx
         for l in range(self.L):
             if evs is not None:
                 evs[l][0].record()
-            c.attn_prefill(self.q[l] if q is None else q, self.k[l] if k is None else k,
-                           self.v[l] if v is None else v, self.o if o is None else o, self.scale,
-                           layer_mode=mode, layer=l, row_ptr=row_ptr, col=col, block=BLOCK,
-                           stream=stream)
+            c.attn_prefill(self.q[l], self.k[l], self.v[l], self.o, self.scale, layer_mode=mode,
+                           layer=l, row_ptr=row_ptr, col=col, block=BLOCK)
             if evs is not None:
                 evs[l][1].record()
 
