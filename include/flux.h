@@ -116,9 +116,12 @@ int flux_selftest_bounded_wait(flux_ctx* ctx, int spin_limit_ms, int* waited_us,
  *   z          = W2 relu(W1 p + b1) + b2;  r = sigmoid(z)
  *   layer_mode [L] uint8 out: 1 (FA) iff r > thresh, else 0 (SA); a tie is SA.
  *   score      [L] fp32 out (optional, may be NULL): r.
- * Uses 4 * (2*Hd + H1) + 64 bytes of the ctx workspace.
+ *   hidden, W1 and W2 start on 16-byte boundaries (they are read in 16-byte
+ *   vectors); b1 and b2 need only fp32 alignment.
+ * Uses 4 * (round_up(2*Hd, 4) + H1) + 64 bytes of the ctx workspace.
  * Errors: INVALID_ARG for null required pointers, sizes <= 0, thresh not
- * finite; SHAPE if the workspace is too small. */
+ * finite, hidden, W1 or W2 not 16-byte aligned; SHAPE if the workspace is
+ * too small. */
 int flux_route(flux_ctx* ctx, const uint16_t* hidden, int T, int Hd, int n_pool,
                const float* W1, const float* b1, int H1,
                const float* W2, const float* b2, int L,

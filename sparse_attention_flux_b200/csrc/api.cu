@@ -388,8 +388,8 @@ int flux_route(flux_ctx* c, const uint16_t* hidden, int T, int Hd, int n_pool, c
     return fail(FLUX_ERR_INVALID_ARG, "flux_route: sizes must be positive");
   if (!(thresh == thresh) || thresh > 3.0e38f || thresh < -3.0e38f)
     return fail(FLUX_ERR_INVALID_ARG, "flux_route: thresh must be finite");
-  if (!aligned16(hidden) || !aligned16(W1))
-    return fail(FLUX_ERR_INVALID_ARG, "flux_route: hidden and W1 must be 16-byte aligned");
+  if (!aligned16(hidden) || !aligned16(W1) || !aligned16(W2))
+    return fail(FLUX_ERR_INVALID_ARG, "flux_route: hidden, W1 and W2 must be 16-byte aligned");
   const size_t need = flux::route_workspace_bytes(Hd, H1);
   if (need > c->workspace_bytes)
     return fail(FLUX_ERR_SHAPE, "flux_route: workspace %zu < %zu bytes", c->workspace_bytes, need);
@@ -408,7 +408,7 @@ int flux_route(flux_ctx* c, const uint16_t* hidden, int T, int Hd, int n_pool, c
   p.layer_mode = layer_mode;
   p.score = score;
   p.pooled = static_cast<float*>(c->workspace);
-  p.hidden1 = p.pooled + 2 * Hd;
+  p.hidden1 = p.pooled + flux::route_hidden1_offset(Hd);
   p.ticket = c->tickets + kMaxTickets;
   const cudaError_t e = flux::launch_route(p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FLUX_OK : cuda_fail(e, "flux_route: launch");

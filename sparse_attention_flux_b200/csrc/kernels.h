@@ -88,6 +88,7 @@ struct RouteLaunch {
   float* hidden1;  // workspace [H1]
   int* ticket;     // workspace, zero between calls
 };
+size_t route_hidden1_offset(int Hd);   // in floats from pooled
 size_t route_workspace_bytes(int Hd, int H1);
 cudaError_t launch_route(const RouteLaunch& p, cudaStream_t stream);
 

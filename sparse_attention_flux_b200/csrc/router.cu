@@ -199,8 +199,13 @@ __global__ void __launch_bounds__(kMlpWarps * 32)
 
 }  // namespace
 
+// hidden1 starts on a 16-byte boundary after pooled[2 Hd]: the last CTA reads
+// it as float4 whenever H1 % 4 == 0, and 2 Hd floats end 8 bytes short of one
+// when Hd is odd.
+size_t route_hidden1_offset(int Hd) { return static_cast<size_t>(2 * Hd + 3) & ~static_cast<size_t>(3); }
+
 size_t route_workspace_bytes(int Hd, int H1) {
-  return static_cast<size_t>(2 * Hd + H1) * sizeof(float) + 64;
+  return (route_hidden1_offset(Hd) + static_cast<size_t>(H1)) * sizeof(float) + 64;
 }
 
 cudaError_t launch_route(const RouteLaunch& p, cudaStream_t stream) {

@@ -85,3 +85,40 @@ def test_route_twice_in_a_row_is_stable(ctx):
     a = _run(ctx, hidden, W1, b1, W2, b2, 0.5)
     b = _run(ctx, hidden, W1, b1, W2, b2, 0.5)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("T,Hd,H1,L,n_pool", [
+    (4096, 64, 32, 4, 104),        # the most rows whose loads the pool issues at once
+    (4096, 64, 32, 4, 105),        # one more: the pool's row loop
+    (4096, 256, 64, 6, 400),       # a wider pooling window than the pages' 100
+    (333, 17, 7, 3, 100),          # odd Hd: scalar pool and W1 dot; H1 % 4 != 0: scalar W2
+    (333, 17, 8, 3, 100),          # odd Hd with float4 W2: hidden1 after 34 pooled floats
+    (512, 3072, 36, 5, 100),       # in_dim 6144: W1 streamed rather than held ahead
+    (512, 2562, 130, 9, 100),      # in_dim 5124: just past the held W1 slice
+])
+def test_route_every_kernel_path(ctx, T, Hd, H1, L, n_pool):
+    hidden, W1, b1, W2, b2 = synth.router_inputs(T, Hd, H1, L, synth.seed_for(0, salt=Hd + n_pool),
+                                                 coin_bias=2.0)
+    mode_o, z, r = oracle.route(hidden, W1, b1, W2, b2, 0.5, n_pool=n_pool)
+    mode_g, score_g = _run(ctx, hidden, W1, b1, W2, b2, 0.5, n_pool=n_pool)
+    assert np.array_equal(mode_g, mode_o), (mode_g, mode_o, z)
+    np.testing.assert_allclose(score_g, r, rtol=0, atol=2e-6)
+    assert np.abs(z).min() > 1e-5
+
+
+def test_route_rejects_misaligned_weights(ctx):
+    """W1 and W2 are read in 16-byte vectors; a view 4 bytes off is refused on the host."""
+    hidden, W1, b1, W2, b2 = synth.router_inputs(64, 16, 8, 2, 5)
+    dev = ctx.device
+    mode = torch.zeros(2, dtype=torch.uint8, device=dev)
+    args = dict(hidden=synth.torch_from_bits(hidden).to(dev), W1=torch.from_numpy(W1).to(dev),
+                b1=torch.from_numpy(b1).to(dev), W2=torch.from_numpy(W2).to(dev),
+                b2=torch.from_numpy(b2).to(dev))
+    for name in ("W1", "W2"):
+        t = args[name]
+        off = torch.empty(t.numel() + 1, dtype=torch.float32, device=dev)[1:].view(t.shape)
+        off.copy_(t)
+        bad = dict(args, **{name: off})
+        with pytest.raises(FluxError):
+            ctx.route(bad["hidden"], bad["W1"], bad["b1"], bad["W2"], bad["b2"], 0.5, mode)
+    ctx.check()

@@ -1,9 +1,10 @@
 """The prefill softmax takes exponentials against the running max and redoes a tile
 only when its row sum passes 2^20.  These cases drive that path hard and compare
 with the oracle: scores that climb steadily along the keys (the running max goes
-stale by tens of log2 units per tile), one key far above the rest (P overflows to
-infinity in the first pass and must be caught), and SA without sink blocks, where a
-row's first tiles can be fully masked."""
+stale by tens of log2 units per tile), one key far above the rest at several
+positions within a tile (P overflows to infinity in the first pass and must be
+caught), and SA without sink blocks, where a row's first tiles can be fully
+masked."""
 import math
 
 import numpy as np
@@ -69,23 +70,32 @@ def test_scores_climbing_along_the_keys(ctx, rate, mode):
     assert_close_lse(lse, rl, f"climbing lse rate {rate} mode {mode}")
 
 
+@pytest.mark.parametrize("row,key", [
+    (1023, 984),    # key 88 of the row's last tile
+    (1023, 901),    # key 5: the tile's first 32-key chunk
+    (1023, 996),    # key 100: its last chunk
+    (1023, 1023),   # the diagonal key, the tile's last
+    (520, 500),     # key 116 of a middle tile, with more tiles after it
+])
 @pytest.mark.parametrize("mode", [1, 0])
-def test_one_key_far_above_the_rest(ctx, mode):
-    # One key in the last tile scores ~250 log2 units above everything before it: the
-    # first pass's exponentials overflow to infinity and the tile must be redone.
+def test_one_key_far_above_the_rest(ctx, mode, row, key):
+    # One key scores ~250 log2 units above everything before it in one query row: the
+    # exponentials against the running max overflow to infinity and the tile must be
+    # redone with O and l rescaled.
     T, Hq, Hkv, d = 1024, 2, 1, 128
     q, k, v = synth.attention_inputs(1, T, Hq, Hkv, d, seed=77)
     qf = synth.bf16_bits_to_f32(q)
     kf = synth.bf16_bits_to_f32(k)
-    u = T - 40
-    # align key u with query row T-1 of head 0, scaled so its score is ~ +180 natural units
-    qrow = qf[0, T - 1, 0]
-    kf[0, u, 0] = qrow / np.dot(qrow, qrow) * 180.0 / (1 / math.sqrt(d))
+    # align the key with query row `row` of head 0, scaled so its score is ~ +180 natural units
+    qrow = qf[0, row, 0]
+    kf[0, key, 0] = qrow / np.dot(qrow, qrow) * 180.0 / (1 / math.sqrt(d))
     k = synth.to_bf16_bits(kf)
     o, lse, ro, rl = _run(ctx, q, k, v, 1 / math.sqrt(d), mode)
     assert np.isfinite(lse).all()
-    assert_close_attn(o, ro, f"one far key mode {mode}")
-    assert_close_lse(lse, rl, f"one far key lse mode {mode}")
+    assert_close_attn(o, ro, f"far key {key} row {row} mode {mode}")
+    assert_close_lse(lse, rl, f"far key {key} row {row} lse mode {mode}")
+    # the row is (nearly) the far key's value row
+    assert rl[0, 0, row] > 170.0
 
 
 def test_sa_without_sink_blocks(ctx):
