@@ -155,6 +155,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   // the split partials and merge tickets of a shared workspace), so it waits
   // for that kernel first; what overlaps is the launch and the CTA dispatch.
   griddep_launch_dependents();
+  // This CTA's own barriers and the tensor-map descriptors (launch parameters)
+  // owe nothing to the previous kernel: they are set up while it finishes.
+  if (tid == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kComputeWarps);
+    }
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
   griddep_wait();
   const int G = a.Hq / a.Hkv;   // 1..kMaxGroup, checked on the host
   // Per-head routing: the group reads the FA range if any of its heads is FA;
@@ -187,14 +198,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
 
-  if (tid == 0) {
-    for (int st = 0; st < kStages; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&empty[st], kComputeWarps);
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();
+  __syncthreads();   // the barriers initialised above are visible to every warp
 
   const int gq = lane >> 2, tq = lane & 3;   // fragment row (head) and column pair
   float m_run = -INFINITY, l_part = 0.f;
@@ -227,8 +231,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncwarp();
     }
     if (lane == 0 && ntiles > 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       int issued = 0;
       for (int k = 0; k < ntiles; ++k) {
         const int st = k % kStages;
@@ -481,10 +483,13 @@ void decode_plan(int B, int Hkv, int S_max, int sink_blocks, int window_blocks, 
   const long long one_wave = std::max<long long>(1, slots / groups);
   sa_splits = std::max<long long>(1, std::min(sa_splits, one_wave));
   if (sa_splits > sa_tiles) sa_splits = std::max<long long>(1, sa_tiles);
-  const long long tsa = sa_tiles > 0 ? (sa_tiles + sa_splits - 1) / sa_splits : 1;
+  long long tsa = sa_tiles > 0 ? (sa_tiles + sa_splits - 1) / sa_splits : 1;
   const long long need_sa = (sa_tiles + tsa - 1) / tsa;
   ns = static_cast<int>(std::max<long long>(ns, need_sa));
-  if (ns > 65535) ns = 65535;   // grid z limit; the chunks grow instead
+  if (ns > 65535) {   // grid z limit (not reached: both plans stay within a wave or two)
+    ns = 65535;       // the FA chunks and the SA tiles per split grow instead
+    tsa = std::max<long long>(tsa, (sa_tiles + ns - 1) / ns);
+  }
   int cfa = (S_max + ns - 1) / ns;
   cfa = ((cfa + kTok - 1) / kTok) * kTok;
   if (cfa < kTok) cfa = kTok;

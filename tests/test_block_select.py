@@ -81,6 +81,28 @@ def test_scores_and_mask_match_oracle(ctx, case):
     print(f"{case}: {open_bits} mask bits differ from the oracle pipeline (all open decisions)")
 
 
+@pytest.mark.parametrize("tau", [0.0, 1.0, 2.0])
+def test_tau_edges(ctx, tau):
+    """tau 0 keeps the forced blocks alone (sinks and the diagonal); tau above 1 is
+    never reached, so every causal block is kept; tau 1 is the rounding edge, held to
+    the oracle pipeline with its open decisions."""
+    B, T, Hq, Hkv, d, sink = 1, 1700, 4, 2, 128, 1
+    q, k, _ = synth.attention_inputs(B, T, Hq, Hkv, d, seed=640)
+    mask, score = _select(ctx, q, k, 8, tau, sink)
+    nb = mask.shape[0]
+    lower = np.tril(np.ones((nb, nb), bool))
+    if tau == 0.0:
+        want = np.zeros((nb, nb), np.uint8)
+        want[:, :sink] = 1
+        np.fill_diagonal(want, 1)
+        np.testing.assert_array_equal(mask, want * lower)
+    elif tau == 2.0:
+        np.testing.assert_array_equal(mask, lower.astype(np.uint8))
+    np.testing.assert_array_equal(mask, oracle.select_blocks(score, tau, sink))
+    P = oracle.block_scores(q, k, 128, 8, 1 / math.sqrt(d))
+    _mask_vs_oracle_pipeline(mask, P, list(range(nb)), tau, sink, f"tau {tau}")
+
+
 def test_planted_block_is_selected(ctx):
     # Keys of block 3 are the antidiagonal partners of query block 9's rows times 4:
     # block 3 takes almost all of query block 9's mass, far outside any local window.
