@@ -1,5 +1,5 @@
 """Per-head routing (the contrast case): every query head equals its own FA or SA
-oracle result; uniform head modes equal the layer-level call exactly."""
+oracle result; uniform head modes equal the layer-level call exactly, in prefill and decode."""
 import math
 
 import numpy as np
@@ -49,6 +49,31 @@ def test_prefill_per_head_matches_oracle(ctx, case):
                                 block_mask=oracle.streaming_mask(nb, nb, sink, W), block=block)
     ref = np.where(hm[None, None, :, None] == 1, fa, sa)
     assert_close_attn(bits_of(o), ref, "per-head prefill")
+
+
+@pytest.mark.parametrize("case", [(1, 1000, 8, 2, 128, 128, 1, 3),   # G 4: layer-level uses head pairs
+                                  (2, 300, 6, 2, 64, 64, 0, 2),     # G 3: row pairs in both
+                                  (1, 777, 4, 1, 128, 64, 2, 5)])   # block 64: the CSR map path
+@pytest.mark.parametrize("mode", [1, 0])
+def test_prefill_uniform_head_modes_equal_the_layer_call(ctx, case, mode):
+    """Every head FA (or every head SA) gives exactly the layer-level call's output: each
+    query row meets the same key tiles in the same order; the extra tiles a row-pair unit
+    walks are fully masked for that row, so they add exact zeros."""
+    B, T, Hq, Hkv, d, block, sink, W = case
+    dev = ctx.device
+    q, k, v = synth.attention_inputs(B, T, Hq, Hkv, d, seed=4100 + T + mode)
+    qt, kt, vt = (synth.torch_from_bits(x).to(dev) for x in (q, k, v))
+    rp, col = _index(ctx, T, block, sink, W)
+    scale = 1 / math.sqrt(d)
+    o_heads = torch.full_like(qt, float("nan"))
+    ctx.attn_prefill_heads(qt, kt, vt, o_heads, scale,
+                           torch.full((Hq,), mode, dtype=torch.uint8, device=dev), rp, col, block)
+    o_layer = torch.full_like(qt, float("nan"))
+    ctx.attn_prefill(qt, kt, vt, o_layer, scale,
+                     layer_mode=torch.tensor([mode], dtype=torch.uint8, device=dev),
+                     row_ptr=rp, col=col, block=block)
+    ctx.check()
+    assert torch.equal(o_heads, o_layer), (o_heads.float() - o_layer.float()).abs().max().item()
 
 
 @pytest.mark.parametrize("pattern", ["mixed", "all_fa", "all_sa", "one_fa_per_group"])
