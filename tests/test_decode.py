@@ -63,6 +63,16 @@ def test_decode_matches_oracle(ctx, case, mode):
     assert_close_lse(lse, rl, "decode lse")
 
 
+def test_no_routing_bits_is_the_fa_path_exactly(ctx):
+    """layer_mode NULL and a routing bit of 1 take the same FA path: identical output and LSE."""
+    B, S_max, seqlens, Hq, Hkv, d, block, sink, W = CASES[1]
+    q, kc, vc = synth.decode_inputs(B, S_max, Hq, Hkv, d, seed=2100)
+    o_none, l_none = _run(ctx, q, kc, vc, seqlens, 0.088, None, sink, W, block)
+    o_fa, l_fa = _run(ctx, q, kc, vc, seqlens, 0.088, 1, sink, W, block)
+    assert np.array_equal(o_none, o_fa)
+    assert np.array_equal(l_none, l_fa)
+
+
 def test_decode_twice_in_a_row_and_mode_switch(ctx):
     # Tickets reset themselves: repeated calls and FA/SA alternation agree.
     B, S_max, Hq, Hkv, d = 2, 3000, 8, 2, 128

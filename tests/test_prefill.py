@@ -107,6 +107,16 @@ def test_routing_bit_is_read_on_device(ctx):
     assert_close_attn(o_sa, ro, "SA")
 
 
+def test_no_routing_bits_is_the_fa_path_exactly(ctx):
+    """layer_mode NULL and a routing bit of 1 take the same FA path: identical output and LSE."""
+    B, T, Hq, Hkv, d = 2, 777, 8, 2, 128
+    q, k, v = synth.attention_inputs(B, T, Hq, Hkv, d, seed=57)
+    o_none, l_none = _run(ctx, q, k, v, 0.09, None)
+    o_fa, l_fa = _run(ctx, q, k, v, 0.09, 1)
+    assert np.array_equal(o_none, o_fa)
+    assert np.array_equal(l_none, l_fa)
+
+
 def test_bad_arguments_are_rejected(ctx):
     q, k, v = synth.attention_inputs(1, 64, 2, 1, 128, seed=1)
     dev = ctx.device
