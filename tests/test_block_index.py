@@ -1,6 +1,5 @@
 """Block mask and compressed block-index list on the GPU: bit-exact against
 the oracle and the hand-enumerated fixture."""
-import os
 
 import numpy as np
 import pytest

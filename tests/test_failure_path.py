@@ -1,8 +1,6 @@
 """Failure detection without a GPU fault: a wait that can never complete gives up after
 its bounded spin limit, the host reads FLUX_ERR_TIMEOUT, and the context keeps working."""
-import math
 
-import numpy as np
 import pytest
 import torch
 

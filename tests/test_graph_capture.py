@@ -3,7 +3,6 @@ FA/SA prefill, KV appends and decode (full cache and ring) give the same bits re
 as run eagerly, and per-step inputs (seqlens) are read at replay time."""
 import math
 
-import numpy as np
 import pytest
 import torch
 

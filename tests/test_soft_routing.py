@@ -2,7 +2,6 @@
 (from flux_route's score output in the end-to-end case)."""
 import math
 
-import numpy as np
 import pytest
 import torch
 
