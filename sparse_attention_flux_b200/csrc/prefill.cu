@@ -346,23 +346,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n > 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t idesc_o = umma_idesc_bf16(kBM, D, false, true);
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // Base descriptors are built once; a k-step or a ring slot adds its byte
+      // offset / 16 to the 14-bit start-address field (shared memory is below
+      // 256 KB, so the field never carries).  The MMA issue path then does one
+      // 64-bit add per operand, which shortens both the issuing thread's loop
+      // and the PV / next-S MMAs on the softmax's round trip.
+      const uint64_t dq0 = umma_smem_desc(smem_u32(sQ), 16, 1024, kSwizzle128B);
+      const uint64_t dk0 = umma_smem_desc(smem_u32(sK), 16, 1024, kSwizzle128B);
+      const uint64_t dv0 = umma_smem_desc(smem_u32(sV), kChunkBytes, 1024, kSwizzle128B);
+      constexpr uint64_t kSlot = static_cast<uint64_t>((CH * kChunkBytes) >> 4);
       auto issue_s = [&](int i, int s) {
-        const uint32_t qb = q_addr + i * CH * kChunkBytes, kb = k_addr + s * CH * kChunkBytes;
+        const uint64_t a0 = dq0 + (i ? kSlot : 0), b0 = dk0 + (s ? kSlot : 0);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
-          umma_bf16_ss(tmem + i * 128, umma_smem_desc(qb + off, 16, 1024, kSwizzle128B),
-                       umma_smem_desc(kb + off, 16, 1024, kSwizzle128B), idesc_s, ks > 0);
+          const uint64_t off = static_cast<uint64_t>(((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4);
+          umma_bf16_ss(tmem + i * 128, a0 + off, b0 + off, idesc_s, ks > 0);
         }
       };
       auto issue_pv = [&](int i, int s, bool acc) {
-        const uint32_t vb = v_addr + s * CH * kChunkBytes;
+        const uint64_t b0 = dv0 + (s ? kSlot : 0);
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks)
           umma_bf16_ts(tmem + 256 + i * 128, tmem + i * 128 + ks * 8,
-                       umma_smem_desc(vb + ks * 16 * 128, kChunkBytes, 1024, kSwizzle128B),
-                       idesc_o, (acc || ks > 0) ? 1u : 0u);
+                       b0 + static_cast<uint64_t>((ks * 16 * 128) >> 4), idesc_o,
+                       (acc || ks > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&bars[B_Q], 0, a.st) && mbar_wait(&bars[B_KF], 0, a.st);
       if (ok) {
